@@ -1,0 +1,369 @@
+#!/usr/bin/env python
+"""Benchmark of one absorbed-MLA decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload long] [--impl reference]
+
+A step is one pass of the whole path over one batch: append the batch's new
+cache rows, absorb the queries, split-KV attention, combine, up-project.  The
+default workload is the long-context one (8 sequences x 131072 cached rows,
+128 heads, bf16 paged cache, 64 splits of 2048 rows); its 1.21 GB cache is
+larger than L2, so successive steps stream it from HBM.
+
+Rank 0 prints one JSON line.  Under torchrun each rank runs the same workload
+on its own GPU (independent sequences, no data-path collective: weak scaling);
+time is the max over ranks.  `--impl reference` times the CPU fp64 oracle
+instead, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "MLA decode tokens/s, latent-cache HBM GB/s and % of B200 roofline"
+CACHE_BYTES = {"f32": 2304, "bf16": 1152, "e4m3": 580}   # per cached row: 576 numbers (+ fp32 scale)
+DECODE_SRC = ["latent_attention_decode_absorbed_b200/csrc/decode_simt.cu"]
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_traffic.md")
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def decode_src_hash():
+    h = hashlib.sha256()
+    for f in DECODE_SRC:
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload):
+    """DRAM bytes per decode launch from the committed ncu summary, if it was
+    taken on the current decode kernel source for this workload."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    src = decode_src_hash()
+    for line in open(TRAFFIC_FILE):
+        m = re.match(r"\s*-?\s*traffic_per_launch\s+workload=(\S+)\s+src=(\S+)\s+bytes=(\d+)", line)
+        if m and m.group(1) == workload and m.group(2) == src:
+            return int(m.group(3))
+    return None
+
+
+def algorithmic(w, lens):
+    rows = int(lens.sum())
+    bytes_ = rows * CACHE_BYTES[w.cache_dtype]
+    vis = sum(int(L) - w.q_len + t + 1 for L in lens for t in range(w.q_len))  # rows seen, all queries
+    flops = 2.0 * w.n_heads * vis * (576 + 512)
+    return bytes_, flops
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = os.path.join("/tmp", f"mla_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu_id), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0])); smax = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def gpu_smi_id(dev_index):
+    import torch
+    try:
+        p = torch.cuda.get_device_properties(dev_index)
+        return f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+    except Exception:
+        return dev_index
+
+
+# ------------------------------------------------------------------ CPU oracle timing
+def time_oracle(w, heads, budget_s, min_reps=1):
+    """Time the fp64 oracle's absorbed step for sequence 0's query rows over
+    its full cache, restricted to `heads` heads; repeat up to budget_s.
+    The cache (RMSNorm/RoPE of every row) is state built before timing, as on
+    the GPU.  Returns (query tokens per second, reps, seconds, cores)."""
+    import oracle
+    kv = W.kv_rows(w, 0)
+    c_hat, k_r = oracle.sequence_cache(kv, w.cache_dtype, None, w.eps, w.theta)
+    qn, qp = W.queries(w)
+    wuk, wuv = W.weights(w)
+    hs = slice(0, heads)
+    qn, qp = qn[:w.q_len, hs], qp[:w.q_len, hs]
+    wuk, wuv = wuk[hs], wuv[hs]
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.attention_absorbed(qn, qp, wuk, wuv, c_hat, k_r)
+        reps += 1
+        el = time.perf_counter() - t0
+        if reps >= min_reps and el >= budget_s:
+            break
+        if reps >= min_reps and el * (reps + 1) / reps > 3 * budget_s:
+            break
+    tokens = reps * w.q_len * heads / w.n_heads
+    cores = os.cpu_count()
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max(i.get("num_threads", 1) for i in threadpool_info()) or cores
+    except Exception:
+        pass
+    return tokens / el, reps, el, cores
+
+
+def run_reference(args, w, rank, world):
+    if rank != 0:
+        return 0
+    lens = W.seq_lens(w)
+    heads = min(16, w.n_heads)
+    # one "step" = sequence 0's query rows over its whole cache for `heads` heads
+    import oracle
+    kv = W.kv_rows(w, 0)
+    c_hat, k_r = oracle.sequence_cache(kv, w.cache_dtype, None, w.eps, w.theta)
+    qn, qp = W.queries(w)
+    wuk, wuv = W.weights(w)
+    qn, qp, wuk, wuv = qn[:w.q_len, :heads], qp[:w.q_len, :heads], wuk[:heads], wuv[:heads]
+    for _ in range(args.warmup):
+        oracle.attention_absorbed(qn, qp, wuk, wuv, c_hat, k_r)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.attention_absorbed(qn, qp, wuk, wuv, c_hat, k_r)
+    el = time.perf_counter() - t0
+    tokens = args.steps * w.q_len * heads / w.n_heads
+    value = tokens / el
+    cores = os.cpu_count()
+    sample = (f"sequence 0 of {w.batch}: {w.q_len} query row(s) x {heads} of {w.n_heads} heads over all "
+              f"{int(lens[0])} cached rows per step (= {heads / w.n_heads:.4f} query tokens); absorbed fp64 "
+              f"oracle, cache built before timing")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(w, lens),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w, lens):
+    return {"workload": w.name, "batch": w.batch, "q_len": w.q_len, "n_heads": w.n_heads,
+            "seq_len": int(lens.max()) if w.seq_len else f"U[{w.len_range[0]},{w.len_range[1]}]",
+            "cached_rows": int(lens.sum()), "cache_dtype": w.cache_dtype, "qw_dtype": w.dtype,
+            "paged": w.paged, "page_size": 64, "split_tokens": w.split_tokens,
+            "dims": "d_c=512 d_rope=64 d_nope=128 d_v=128", "parallelism": "replicas (independent sequences per GPU)",
+            "l2": "no flush: the cache is larger than L2" if int(lens.sum()) * CACHE_BYTES[w.cache_dtype] > 256e6
+            else "L2 flushed before every step (256 MB write)"}
+
+
+# ------------------------------------------------------------------ GPU arm
+def run_gpu(args, w, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from workloads.device import DeviceWorkload
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    dw = DeviceWorkload(w, device=dev)
+    step = dw.step
+    lens = dw.lens
+    stream = torch.cuda.current_stream(dev)
+    alg_bytes, alg_flops = algorithmic(w, lens)
+    flush = None
+    if alg_bytes <= 256e6:
+        flush = torch.empty(int(256e6) // 4, dtype=torch.float32, device=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def one_step(ev=None):
+        if flush is not None:
+            flush.fill_(1.0)
+        step.append(dw.kv_new, dw.seq_ids, dw.positions)
+        step.absorb(dw.q_nope, dw.q_pe, dw.w_uk)
+        if ev is not None:
+            ev[0].record(stream)
+        step.attend()
+        if ev is not None:
+            ev[1].record(stream)
+        step.combine()
+        step.project_out(dw.w_uv)
+
+    for _ in range(args.warmup):
+        one_step()
+    torch.cuda.synchronize()
+    assert int(step.err.item()) == 0, "device error flag set"
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(gpu_smi_id(local_rank)) as clk:
+        barrier(); torch.cuda.synchronize()
+        t_start.record(stream)
+        for i in range(args.steps):
+            one_step(evs[i])
+        t_end.record(stream)
+        torch.cuda.synchronize(); barrier()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    decode_ms = [a.elapsed_time(b) for a, b in evs]
+    clocks = clk.summary()
+    # end-to-end through the public API: pinned host inputs in, host output back, every step
+    h_kv = dw.kv_new.cpu().pin_memory()
+    h_qn, h_qp = dw.q_nope.cpu().pin_memory(), dw.q_pe.cpu().pin_memory()
+    h_out = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
+    h2d = h_kv.numel() * h_kv.element_size() + h_qn.numel() * h_qn.element_size() + h_qp.numel() * h_qp.element_size()
+    d2h = h_out.numel() * h_out.element_size()
+
+    def e2e_step():
+        if flush is not None:
+            flush.fill_(1.0)
+        dw.kv_new.copy_(h_kv, non_blocking=True)
+        dw.q_nope.copy_(h_qn, non_blocking=True)
+        dw.q_pe.copy_(h_qp, non_blocking=True)
+        step.run(dw.kv_new, dw.seq_ids, dw.positions, dw.q_nope, dw.q_pe, dw.w_uk, dw.w_uv)
+        h_out.copy_(step.out, non_blocking=True)
+
+    for _ in range(max(3, args.warmup)):
+        e2e_step()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(); torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(); barrier()
+    e2e_ms = e0.elapsed_time(e1)
+    assert int(step.err.item()) == 0, "device error flag set"
+
+    # max over ranks
+    t = torch.tensor([elapsed_ms, e2e_ms, float(np.mean(decode_ms))], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    elapsed_ms, e2e_ms, dec_ms = t.tolist()
+    if rank != 0:
+        return 0
+    tokens_per_step = w.batch * w.q_len
+    value = world * tokens_per_step * args.steps / (elapsed_ms / 1e3)
+    e2e_value = world * tokens_per_step * args.steps / (e2e_ms / 1e3)
+    pk = peaks()
+    achieved = alg_bytes / (dec_ms / 1e3) / 1e9
+    traffic = recorded_traffic(w.name)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
+        "data": "synthetic", "config": workload_config(w, lens),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / pk["hbm_gbs"], "traffic": traffic,
+                     "kernel": "mla_decode_fwd", "peak_source": pk["source"],
+                     "algorithmic_bytes_per_launch": alg_bytes, "launch_ms": dec_ms},
+        "decode": {"cache_gbs": achieved, "tflops": alg_flops / (dec_ms / 1e3) / 1e12,
+                   "tensor_frac_burst": alg_flops / (dec_ms / 1e3) / 1e12 / pk["bf16_tflops"],
+                   "roofline_ms": 1e3 * max(alg_bytes / (pk["hbm_gbs"] * 1e9), alg_flops / (pk["bf16_tflops"] * 1e12)),
+                   "roofline_frac": 1e3 * max(alg_bytes / (pk["hbm_gbs"] * 1e9),
+                                              alg_flops / (pk["bf16_tflops"] * 1e12)) / dec_ms,
+                   "share_of_step": dec_ms / (elapsed_ms / args.steps)},
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": step.LAUNCHES_PER_STEP * args.steps,
+        "clocks": clocks,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        v, reps, el, cores = time_oracle(w, heads=w.n_heads, budget_s=args.cpu_budget)
+        line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                "sample": f"{reps} x sequence 0's {w.q_len} query row(s), all {w.n_heads} heads, "
+                                          f"over {int(lens[0])} cached rows ({el:.1f} s); absorbed fp64 oracle, "
+                                          f"cache built before timing"}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="long", choices=W.WORKLOAD_ORDER)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    w = W.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w, rank, world)
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        return run_gpu(args, w, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,217 @@
+/*
+ * mla.h - C ABI of the B200 (sm_100a) absorbed Multi-head Latent Attention
+ * decode library (libmla.so).
+ *
+ * The library computes one decode step of weight-absorbed MLA attention for
+ * one layer, as defined by the DeepSeek-V2 Appendix C formulas ("DeepSeek-V2:
+ * MLA Explained", section "MLA Full Formulas", parts 2 and 3) with the
+ * absorption of "Optimization Note" on the same page: the key up-projection
+ * W_UK is folded into the query and the value up-projection W_UV is applied
+ * after the softmax sum, so attention runs directly over the cached rows.
+ *
+ * The cache ("KV Compression - DeepSeek-V3", section "How it works") holds one
+ * row of 576 numbers per token: the RMSNorm'd 512-wide joint KV latent c_kv
+ * followed by the 64-wide RoPE'd key k_pe shared by all heads.  Rows live in
+ * pages of `page_size` tokens; a per-sequence block table maps a sequence's
+ * page slot to a page of one pool.
+ *
+ * A decode step for B sequences with T new tokens each, H heads:
+ *   mla_cache_append  new kv_a rows -> cache rows (RMSNorm, RoPE, cast/quantise)
+ *   mla_absorb_q      q_nope, q_pe  -> q_abs = [W_UK^T q_nope ; q_pe]   (576 per head)
+ *   mla_decode_fwd    q_abs, cache  -> split-KV partials (o_part, lse_part)
+ *   mla_combine       partials      -> o_lat (512 per head), lse
+ *   mla_out_uv        o_lat         -> out = W_UV o_lat                 (128 per head)
+ *
+ * Conventions for every entry point
+ *  - Pointers named as device pointers must be device memory (or managed
+ *    memory) of the current device; the caller owns all memory.  No entry
+ *    point allocates, frees or keeps device memory, except the tensor-map
+ *    cache noted at mla_decode_fwd.
+ *  - Tensors are dense, row-major, with the shapes given; device pointers must
+ *    be 16-byte aligned (the cache 128-byte aligned).
+ *  - Calls are asynchronous on `stream`; a return of MLA_OK means the work was
+ *    validated and enqueued.  Argument errors return before anything is
+ *    enqueued.  MLA_ERR_CUDA reports a launch failure (details from
+ *    mla_last_error_message()).  Bad data found on the device (a block-table
+ *    entry outside the pool, a row outside the table) is skipped and recorded
+ *    in `err_word` (when not NULL) as a bitwise OR of MLA_DEVERR_* flags; the
+ *    caller reads it after synchronising.
+ *  - No C++ exception crosses the ABI.  Entry points are thread-safe.
+ */
+#ifndef MLA_H_
+#define MLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Fixed widths of the DeepSeek-V2/V3 attention shape ("KV Compression -
+ * DeepSeek-V3", "How it works"; "DeepSeek-V2: MLA Explained", symbol list). */
+#define MLA_D_C    512   /* joint KV latent width (kv_lora_rank) */
+#define MLA_D_R     64   /* decoupled rope key width (qk_rope_head_dim) */
+#define MLA_D_ROW  576   /* numbers cached per token per layer */
+#define MLA_D_NOPE 128   /* per-head nope query width */
+#define MLA_D_V    128   /* per-head value width */
+#define MLA_PAGE    64   /* the supported page size in tokens */
+#define MLA_MAX_HEADS 128
+
+typedef enum {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_ARG = 1,   /* a null pointer, a bad size or alignment */
+  MLA_ERR_UNSUPPORTED = 2,   /* a valid but unsupported dtype / shape combination */
+  MLA_ERR_CUDA = 3,          /* a CUDA runtime error while enqueuing */
+  MLA_ERR_BAD_INDEX = 4,     /* host-checked index out of range */
+  MLA_ERR_TIMEOUT = 5        /* a device wait ran out (reported via err_word) */
+} mla_status;
+
+typedef enum {
+  MLA_F32 = 0,
+  MLA_BF16 = 1,
+  MLA_E4M3 = 2               /* OCP FP8 E4M3 (cache only), one fp32 scale per token */
+} mla_dtype;
+
+/* Device error flags OR-ed into err_word. */
+#define MLA_DEVERR_PAGE     0x1  /* block-table entry < 0 or >= num_pages: row skipped */
+#define MLA_DEVERR_POSITION 0x2  /* append position/sequence outside the table: row skipped */
+#define MLA_DEVERR_TIMEOUT  0x4  /* a bounded device wait gave up: results invalid */
+
+/* Short static string for a status code; never NULL. */
+const char* mla_status_string(int status);
+
+/* Detail of the last non-OK status returned on the calling thread ("" if none). */
+const char* mla_last_error_message(void);
+
+/* Library version: major*10000 + minor*100 + patch. */
+int mla_version(void);
+
+/*
+ * mla_rope_table (host function, no GPU needed)
+ * RoPE rotation table for the decoupled key ("DeepSeek-V2: MLA Explained",
+ * "MLA Full Formulas" part 2, k^R_t = RoPE(W^KR h_t)).  Pair i (channels 2i,
+ * 2i+1) of a row at position p turns by angle p * theta^(-2i/64); the angle,
+ * cos and sin are evaluated in double precision and rounded to float.
+ *   theta         rotary base (> 1), e.g. 10000
+ *   max_pos       number of positions (>= 1)
+ *   cos_out, sin_out  HOST arrays [max_pos, 32] float, caller-owned
+ * Returns MLA_ERR_INVALID_ARG for null pointers or bad sizes.
+ */
+mla_status mla_rope_table(double theta, int max_pos, float* cos_out, float* sin_out);
+
+/*
+ * mla_cache_append
+ * Writes the cache rows of new tokens ("KV Compression - DeepSeek-V3", "How it
+ * works" and "Official code": split the 576-wide wkv_a output [512, 64],
+ * RMSNorm the latent, RoPE the rope part, store both; "DeepSeek-V2: MLA
+ * Explained", "Caching Strategy").  For new token n:
+ *   c   = kv_a[n, 0:512],  cache_c = c / sqrt(mean(c^2) + eps) * norm_gain
+ *   k   = kv_a[n, 512:576], cache_k[2i] = k[2i] cos - k[2i+1] sin,
+ *                           cache_k[2i+1] = k[2i] sin + k[2i+1] cos  (table row positions[n])
+ *   row = [cache_c ; cache_k] stored at
+ *         cache[(block_table[seq_ids[n], positions[n] / page_size] * page_size
+ *                + positions[n] % page_size) * 576 ...]
+ *   E4M3 cache: a = max|row|, cache_scale[slot] = a / 448,
+ *         codes = e4m3_rne_satfinite(row * (448 / a)); a = 0 stores zeros and scale 0.
+ * Arithmetic is fp32.
+ *   kv_a        device [n_new, 576], kv_dtype F32 or BF16
+ *   seq_ids     device int32 [n_new], each in [0, batch)
+ *   positions   device int32 [n_new], each in [0, max_pages_per_seq*page_size) and < rope_max_pos
+ *   block_table device int32 [batch, max_pages_per_seq], entries in [0, num_pages)
+ *   norm_gain   device float [512] or NULL (gain 1)
+ *   eps         RMSNorm epsilon (>= 0)
+ *   rope_cos, rope_sin device float [rope_max_pos, 32] (see mla_rope_table)
+ *   cache       device [num_pages, page_size, 576] of cache_dtype (F32, BF16, E4M3)
+ *   cache_scale device float [num_pages, page_size] for E4M3, else ignored (may be NULL)
+ *   err_word    device int32 or NULL; rows whose sequence, position or page is out of
+ *               range are skipped and flagged (MLA_DEVERR_POSITION / MLA_DEVERR_PAGE)
+ * Rows with the same (sequence, position) in one call race; distinct slots never do.
+ */
+mla_status mla_cache_append(const void* kv_a, mla_dtype kv_dtype, int n_new,
+                            const int32_t* seq_ids, const int32_t* positions,
+                            const int32_t* block_table, int batch, int max_pages_per_seq,
+                            int page_size, const float* norm_gain, float eps,
+                            const float* rope_cos, const float* rope_sin, int rope_max_pos,
+                            void* cache, float* cache_scale, mla_dtype cache_dtype,
+                            int num_pages, int32_t* err_word, cudaStream_t stream);
+
+/*
+ * mla_absorb_q
+ * Absorbed query ("DeepSeek-V2: MLA Explained", "Optimization Note": W_UK
+ * merged into the query; "MLA Full Formulas" part 1, q_{t,i} = [q^C; q^R]):
+ *   q_abs[r, h, 0:512]   = sum_k W_UK[h, k, :] * q_nope[r, h, k]     (fp32 accumulate)
+ *   q_abs[r, h, 512:576] = q_pe[r, h, :]
+ *   q_nope device [rows, n_heads, 128], q_pe device [rows, n_heads, 64],
+ *   w_uk   device [n_heads, 128, 512], q_abs device [rows, n_heads, 576]; all of `dtype`
+ *   (F32 or BF16).  rows >= 1, 1 <= n_heads <= 128.
+ */
+mla_status mla_absorb_q(const void* q_nope, const void* q_pe, const void* w_uk, void* q_abs,
+                        int rows, int n_heads, mla_dtype dtype, cudaStream_t stream);
+
+/*
+ * mla_decode_fwd
+ * Split-KV attention over the cache in latent space ("DeepSeek-V2: MLA
+ * Explained", "MLA Full Formulas" part 3 with the absorption of
+ * "Optimization Note").  For sequence b with seq_lens[b] = L_b cached rows
+ * (the step's q_len new rows included), query t (row r = b*q_len + t) sits at
+ * position L_b - q_len + t and sees rows j <= L_b - q_len + t.  Split s covers
+ * rows [s*split_tokens, (s+1)*split_tokens).  For each (r, h, s):
+ *   z_j = softmax_scale * (q_abs[r,h,0:512] . c_j + q_abs[r,h,512:576] . k_j)
+ *         (E4M3 cache: c_j, k_j are codes times cache_scale[j])
+ *   o_part[r,h,s,:] = sum_j e^{z_j - m} c_j / sum_j e^{z_j - m}   over the split's visible j
+ *   lse_part[r,h,s] = m + ln sum_j e^{z_j - m}  (natural log; -inf and o = 0 for an empty split)
+ *   q_abs       device [batch*q_len, n_heads, 576], q_dtype F32 or BF16
+ *   cache       device [num_pages, page_size, 576]; cache_scale as for mla_cache_append
+ *   block_table device int32 [batch, max_pages_per_seq]
+ *   seq_lens    device int32 [batch], q_len <= L_b <= max_pages_per_seq*page_size
+ *   num_splits * split_tokens must cover the longest sequence; split_tokens is
+ *               a positive multiple of page_size
+ *   o_part      device float [batch*q_len, n_heads, num_splits, 512]   (caller-owned workspace)
+ *   lse_part    device float [batch*q_len, n_heads, num_splits]
+ *   err_word    device int32 or NULL (MLA_DEVERR_PAGE, MLA_DEVERR_TIMEOUT)
+ * Supported: page_size 64; q_dtype F32 with cache F32; q_dtype BF16 with cache
+ * BF16 or E4M3.  BF16/E4M3 run on the tcgen05 tensor cores (bf16 operands,
+ * fp32 accumulation); F32 runs exact fp32 on the CUDA cores.  The library
+ * caches TMA descriptors per (cache pointer, pool size) on the host.
+ */
+mla_status mla_decode_fwd(const void* q_abs, mla_dtype q_dtype, const void* cache,
+                          const float* cache_scale, mla_dtype cache_dtype, int num_pages,
+                          const int32_t* block_table, int max_pages_per_seq, int page_size,
+                          const int32_t* seq_lens, int batch, int q_len, int n_heads,
+                          int num_splits, int split_tokens, float softmax_scale,
+                          float* o_part, float* lse_part, int32_t* err_word,
+                          cudaStream_t stream);
+
+/*
+ * mla_combine
+ * Log-sum-exp merge of split partials (the softmax sum of "MLA Full Formulas"
+ * part 3 decomposed over disjoint row ranges):
+ *   M = max_s lse_part[r,h,s];  w_s = e^{lse_s - M}  (0 for lse_s = -inf)
+ *   o_lat[r,h,:] = sum_s w_s o_part[r,h,s,:] / sum_s w_s,   lse_out[r,h] = M + ln sum_s w_s
+ *   o_part device float [rows, n_heads, num_splits, 512], lse_part [rows, n_heads, num_splits]
+ *   o_lat  device [rows, n_heads, 512] of o_dtype (F32 or BF16)
+ *   lse_out device float [rows, n_heads] or NULL
+ */
+mla_status mla_combine(const float* o_part, const float* lse_part, int rows, int n_heads,
+                       int num_splits, void* o_lat, mla_dtype o_dtype, float* lse_out,
+                       cudaStream_t stream);
+
+/*
+ * mla_out_uv
+ * Value up-projection applied after the softmax sum ("DeepSeek-V2: MLA
+ * Explained", "MLA Full Formulas" part 2, v^C = W^UV c, moved past the sum per
+ * "Optimization Note"):
+ *   out[r, h, i] = sum_c W_UV[h, i, c] * o_lat[r, h, c]    (fp32 accumulate)
+ *   o_lat device [rows, n_heads, 512], w_uv device [n_heads, 128, 512],
+ *   out device [rows, n_heads, 128]; all of `dtype` (F32 or BF16).
+ */
+mla_status mla_out_uv(const void* o_lat, const void* w_uv, void* out, int rows, int n_heads,
+                      mla_dtype dtype, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_H_ */

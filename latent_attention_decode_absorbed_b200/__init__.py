@@ -1,0 +1,142 @@
+"""Python binding of libmla.so, the sm_100a absorbed-MLA decode library.
+
+Argument marshalling only: every function forwards to the C entry point of
+the same name in ``include/mla.h`` and raises ``MlaError`` on a non-OK
+status.  Tensor arguments are torch tensors (their device pointers are
+passed); PyTorch supplies device memory and streams, nothing else.  There is
+no CPU fallback: if the shared library is missing, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmla.so")
+
+MLA_OK, MLA_ERR_INVALID_ARG, MLA_ERR_UNSUPPORTED, MLA_ERR_CUDA, MLA_ERR_BAD_INDEX, MLA_ERR_TIMEOUT = range(6)
+MLA_F32, MLA_BF16, MLA_E4M3 = 0, 1, 2
+MLA_DEVERR_PAGE, MLA_DEVERR_POSITION, MLA_DEVERR_TIMEOUT = 0x1, 0x2, 0x4
+D_C, D_R, D_ROW, D_NOPE, D_V, PAGE = 512, 64, 576, 128, 128, 64
+
+# entry points with their ctypes signatures (p = pointer, i = int, f = float, d = double)
+_SIGS = {
+    "mla_status_string": ("s", "i"),
+    "mla_last_error_message": ("s", ""),
+    "mla_version": ("i", ""),
+    "mla_rope_table": ("i", "dipp"),
+    "mla_cache_append": ("i", "piipppiiipfppippiipp"),
+    "mla_absorb_q": ("i", "ppppiiip"),
+    "mla_decode_fwd": ("i", "pippiipiipiiiiifpppp"),
+    "mla_combine": ("i", "ppiiipipp"),
+    "mla_out_uv": ("i", "pppiiip"),
+}
+_CT = {"p": ctypes.c_void_p, "i": ctypes.c_int, "f": ctypes.c_float, "d": ctypes.c_double,
+       "s": ctypes.c_char_p}
+
+_lib = None
+
+
+class MlaError(RuntimeError):
+    def __init__(self, fn, status, msg):
+        super().__init__(f"{fn}: status {status} ({status_string(status)}): {msg}")
+        self.status = status
+
+
+def lib():
+    """Load libmla.so (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libmla.so not built at {LIB_PATH}; run "
+                               "`python -m latent_attention_decode_absorbed_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            f = getattr(L, name)
+            f.restype = _CT[res]
+            f.argtypes = [_CT[c] for c in args]
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().mla_status_string(int(status)).decode()
+
+
+def _ptr(x) -> Optional[int]:
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(fn, status):
+    if status != MLA_OK:
+        raise MlaError(fn, status, lib().mla_last_error_message().decode())
+
+
+def dtype_code(t) -> int:
+    import torch
+    return {torch.float32: MLA_F32, torch.bfloat16: MLA_BF16, torch.uint8: MLA_E4M3,
+            torch.float8_e4m3fn: MLA_E4M3}[t.dtype]
+
+
+def mla_version() -> int:
+    return lib().mla_version()
+
+
+def mla_rope_table(theta: float, max_pos: int, cos_out, sin_out):
+    """Host tables [max_pos, 32] float32 (numpy arrays or CPU tensors)."""
+    cp = cos_out.ctypes.data if hasattr(cos_out, "ctypes") else cos_out.data_ptr()
+    sp = sin_out.ctypes.data if hasattr(sin_out, "ctypes") else sin_out.data_ptr()
+    _check("mla_rope_table", lib().mla_rope_table(float(theta), int(max_pos), cp, sp))
+
+
+def mla_cache_append(kv_a, kv_dtype, n_new, seq_ids, positions, block_table, batch, max_pages_per_seq,
+                     page_size, norm_gain, eps, rope_cos, rope_sin, rope_max_pos, cache, cache_scale,
+                     cache_dtype, num_pages, err_word=None, stream=None):
+    _check("mla_cache_append", lib().mla_cache_append(
+        _ptr(kv_a), int(kv_dtype), int(n_new), _ptr(seq_ids), _ptr(positions), _ptr(block_table),
+        int(batch), int(max_pages_per_seq), int(page_size), _ptr(norm_gain), float(eps), _ptr(rope_cos),
+        _ptr(rope_sin), int(rope_max_pos), _ptr(cache), _ptr(cache_scale), int(cache_dtype),
+        int(num_pages), _ptr(err_word), _stream(stream)))
+
+
+def mla_absorb_q(q_nope, q_pe, w_uk, q_abs, rows, n_heads, dtype, stream=None):
+    _check("mla_absorb_q", lib().mla_absorb_q(_ptr(q_nope), _ptr(q_pe), _ptr(w_uk), _ptr(q_abs),
+                                              int(rows), int(n_heads), int(dtype), _stream(stream)))
+
+
+def mla_decode_fwd(q_abs, q_dtype, cache, cache_scale, cache_dtype, num_pages, block_table,
+                   max_pages_per_seq, page_size, seq_lens, batch, q_len, n_heads, num_splits,
+                   split_tokens, softmax_scale, o_part, lse_part, err_word=None, stream=None):
+    _check("mla_decode_fwd", lib().mla_decode_fwd(
+        _ptr(q_abs), int(q_dtype), _ptr(cache), _ptr(cache_scale), int(cache_dtype), int(num_pages),
+        _ptr(block_table), int(max_pages_per_seq), int(page_size), _ptr(seq_lens), int(batch),
+        int(q_len), int(n_heads), int(num_splits), int(split_tokens), float(softmax_scale),
+        _ptr(o_part), _ptr(lse_part), _ptr(err_word), _stream(stream)))
+
+
+def mla_combine(o_part, lse_part, rows, n_heads, num_splits, o_lat, o_dtype, lse_out=None, stream=None):
+    _check("mla_combine", lib().mla_combine(_ptr(o_part), _ptr(lse_part), int(rows), int(n_heads),
+                                            int(num_splits), _ptr(o_lat), int(o_dtype), _ptr(lse_out),
+                                            _stream(stream)))
+
+
+def mla_out_uv(o_lat, w_uv, out, rows, n_heads, dtype, stream=None):
+    _check("mla_out_uv", lib().mla_out_uv(_ptr(o_lat), _ptr(w_uv), _ptr(out), int(rows), int(n_heads),
+                                          int(dtype), _stream(stream)))
+
+
+from .step import DecodeStep  # noqa: E402,F401

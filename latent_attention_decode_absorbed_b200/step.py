@@ -1,0 +1,105 @@
+"""One layer's decode step over a paged latent cache, as five library calls.
+
+``DecodeStep`` owns the device buffers of one layer (cache, page table,
+rope tables, workspace and outputs, as torch tensors) and runs
+
+    mla_cache_append -> mla_absorb_q -> mla_decode_fwd -> mla_combine -> mla_out_uv
+
+on one stream.  It only allocates and marshals; every step runs in libmla.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+from . import (D_C, D_R, D_ROW, D_V, MLA_BF16, MLA_E4M3, MLA_F32, PAGE, mla_absorb_q, mla_cache_append,
+               mla_combine, mla_decode_fwd, mla_out_uv, mla_rope_table)
+
+_DT = {"f32": MLA_F32, "bf16": MLA_BF16, "e4m3": MLA_E4M3}
+
+
+def _torch_dtype(code):
+    import torch
+    return {MLA_F32: torch.float32, MLA_BF16: torch.bfloat16, MLA_E4M3: torch.uint8}[code]
+
+
+class DecodeStep:
+    """Device state of one layer for `batch` sequences with `q_len` new tokens.
+
+    block_table: int32 [batch, max_pages] (host array or tensor); num_pages:
+    size of the page pool; split_tokens: split-KV chunk (multiple of 64)."""
+
+    def __init__(self, *, batch, q_len, n_heads, dtype, cache_dtype, block_table, num_pages,
+                 split_tokens, max_pos=None, theta=10000.0, eps=1e-6, norm_gain=None,
+                 softmax_scale=None, device="cuda"):
+        import torch
+        self.torch = torch
+        self.batch, self.q_len, self.n_heads = int(batch), int(q_len), int(n_heads)
+        self.dtype, self.cache_dtype = _DT[dtype], _DT[cache_dtype]
+        self.device = torch.device(device)
+        bt = torch.as_tensor(np.asarray(block_table, dtype=np.int32))
+        self.block_table = bt.to(self.device)
+        self.max_pages = int(bt.shape[1])
+        self.num_pages = int(num_pages)
+        self.split_tokens = int(split_tokens)
+        self.num_splits = int(math.ceil(self.max_pages * PAGE / self.split_tokens))
+        self.eps = float(eps)
+        self.softmax_scale = float(softmax_scale if softmax_scale is not None else 1.0 / math.sqrt(192.0))
+        self.max_pos = int(max_pos if max_pos is not None else self.max_pages * PAGE)
+        cos = np.empty((self.max_pos, D_R // 2), np.float32)
+        sin = np.empty_like(cos)
+        mla_rope_table(theta, self.max_pos, cos, sin)
+        self.rope_cos = torch.from_numpy(cos).to(self.device)
+        self.rope_sin = torch.from_numpy(sin).to(self.device)
+        self.norm_gain = None if norm_gain is None else torch.as_tensor(
+            np.asarray(norm_gain, np.float32)).to(self.device)
+        dev = self.device
+        self.cache = torch.empty((self.num_pages, PAGE, D_ROW), dtype=_torch_dtype(self.cache_dtype), device=dev)
+        self.cache_scale = (torch.zeros((self.num_pages, PAGE), dtype=torch.float32, device=dev)
+                            if self.cache_dtype == MLA_E4M3 else None)
+        rows = self.batch * self.q_len
+        qdt = _torch_dtype(self.dtype)
+        self.q_abs = torch.empty((rows, self.n_heads, D_ROW), dtype=qdt, device=dev)
+        self.o_part = torch.empty((rows, self.n_heads, self.num_splits, D_C), dtype=torch.float32, device=dev)
+        self.lse_part = torch.empty((rows, self.n_heads, self.num_splits), dtype=torch.float32, device=dev)
+        self.o_lat = torch.empty((rows, self.n_heads, D_C), dtype=qdt, device=dev)
+        self.lse = torch.empty((rows, self.n_heads), dtype=torch.float32, device=dev)
+        self.out = torch.empty((rows, self.n_heads, D_V), dtype=qdt, device=dev)
+        self.err = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.seq_lens = torch.zeros(self.batch, dtype=torch.int32, device=dev)
+
+    # -- individual calls ------------------------------------------------
+    def append(self, kv_a, seq_ids, positions, stream=None):
+        mla_cache_append(kv_a, _DT["f32"] if kv_a.dtype == self.torch.float32 else MLA_BF16,
+                         kv_a.shape[0], seq_ids, positions, self.block_table, self.batch, self.max_pages,
+                         PAGE, self.norm_gain, self.eps, self.rope_cos, self.rope_sin, self.max_pos,
+                         self.cache, self.cache_scale, self.cache_dtype, self.num_pages, self.err, stream)
+
+    def absorb(self, q_nope, q_pe, w_uk, stream=None):
+        mla_absorb_q(q_nope, q_pe, w_uk, self.q_abs, self.batch * self.q_len, self.n_heads, self.dtype, stream)
+
+    def attend(self, stream=None):
+        mla_decode_fwd(self.q_abs, self.dtype, self.cache, self.cache_scale, self.cache_dtype, self.num_pages,
+                       self.block_table, self.max_pages, PAGE, self.seq_lens, self.batch, self.q_len,
+                       self.n_heads, self.num_splits, self.split_tokens, self.softmax_scale, self.o_part,
+                       self.lse_part, self.err, stream)
+
+    def combine(self, stream=None):
+        mla_combine(self.o_part, self.lse_part, self.batch * self.q_len, self.n_heads, self.num_splits,
+                    self.o_lat, self.dtype, self.lse, stream)
+
+    def project_out(self, w_uv, stream=None):
+        mla_out_uv(self.o_lat, w_uv, self.out, self.batch * self.q_len, self.n_heads, self.dtype, stream)
+
+    # -- the whole step ----------------------------------------------------
+    def run(self, kv_a_new, seq_ids, positions, q_nope, q_pe, w_uk, w_uv, stream=None):
+        """Append the step's new rows, then attend; returns `out` [B*T, H, 128]."""
+        self.append(kv_a_new, seq_ids, positions, stream)
+        self.absorb(q_nope, q_pe, w_uk, stream)
+        self.attend(stream)
+        self.combine(stream)
+        self.project_out(w_uv, stream)
+        return self.out
+
+    LAUNCHES_PER_STEP = 5

@@ -265,14 +265,14 @@ def attention_absorbed(q_nope, q_pe, w_uk, w_uv, c_hat, k_r, softmax_scale=None)
     L = c_hat.shape[0]
     scale = 1.0 / math.sqrt(D_N + D_R) if softmax_scale is None else softmax_scale
     q_lat = absorb_q(q_nope, w_uk)
-    z = (np.einsum("thc,jc->thj", q_lat, c_hat) + np.einsum("thr,jr->thj", q_pe, k_r)) * scale
+    z = ((q_lat.reshape(T * H, D_C) @ c_hat.T + q_pe.reshape(T * H, D_R) @ k_r.T) * scale).reshape(T, H, L)
     for t in range(T):
         z[t, :, L - T + t + 1:] = -np.inf
     m = z.max(axis=-1, keepdims=True)
     e = np.exp(z - m)
     s = e.sum(axis=-1, keepdims=True)
     p = e / s
-    o_lat = np.einsum("thj,jc->thc", p, c_hat)
+    o_lat = (p.reshape(T * H, L) @ c_hat).reshape(T, H, D_C)
     lse = (m + np.log(s))[..., 0]
     out = np.einsum("thc,hvc->thv", o_lat, np.asarray(w_uv, np.float64))
     return out, o_lat, lse
@@ -313,13 +313,17 @@ def attention_partials(q_lat, q_pe, c_hat, k_r, split_tokens: int, num_splits: i
 def combine_partials(o_part, lse_part):
     """Merge split partials: M = max_s lse_s, w_s = exp(lse_s - M),
     o = sum_s w_s o_s / sum_s w_s, lse = M + log sum_s w_s.
+    When no split saw a row (every lse_s = -inf): o = 0, lse = -inf.
     o_part [..., S, 512], lse_part [..., S] -> (o [..., 512], lse [...])."""
     o_part = np.asarray(o_part, np.float64); lse_part = np.asarray(lse_part, np.float64)
     M = lse_part.max(axis=-1, keepdims=True)
-    w = np.where(np.isfinite(lse_part), np.exp(lse_part - M), 0.0)
+    seen = np.isfinite(M)                                  # some split saw a row
+    Ms = np.where(seen, M, 0.0)
+    w = np.where(np.isfinite(lse_part), np.exp(lse_part - Ms), 0.0)
     ws = w.sum(axis=-1, keepdims=True)
-    o = (w[..., None] * o_part).sum(axis=-2) / ws
-    return o, (M + np.log(ws))[..., 0]
+    o = (w[..., None] * o_part).sum(axis=-2) / np.where(seen, ws, 1.0)
+    lse = np.where(seen, Ms + np.log(np.where(seen, ws, 1.0)), -np.inf)
+    return o, lse[..., 0]
 
 
 def out_uv(o_lat, w_uv):

@@ -1,0 +1,89 @@
+"""Whole decode step on the GPU (append -> absorb -> attend -> combine ->
+up-project, through the C ABI) against the fp64 oracle.
+
+Gate: max over (query row, head) of ||out_gpu - out_ref|| / ||out_ref|| over
+the 128-d head output, at most 1e-2 for the bf16 cache, 3e-2 for the e4m3
+cache, 1e-4 for fp32.  The full-size workloads run in the launch
+configuration the benchmark times and are checked on sampled sequences (the
+absorbed oracle for every head, the naive oracle for a few heads)."""
+import numpy as np
+import pytest
+
+import oracle
+import workloads as W
+from gpu_common import TOL, gpu_rows, reference_sequence
+from workloads.device import DeviceWorkload, to_host_f64
+
+pytestmark = pytest.mark.gpu
+torch = pytest.importorskip("torch")
+
+# (workload, sequences checked with the absorbed oracle, (sequence, heads) for the naive oracle)
+FULL = [
+    ("tiny", [0], (0, None)),
+    ("v3_b1", [0], (0, None)),
+    ("serving", [0, 17, 63], (0, [0, 127])),
+    ("long", [0, 7], (0, [0])),
+    ("fp8_mtp", [0, 1, 64, 127], (0, [0, 127])),
+]
+
+SMALL = [
+    W.Workload("ragged_serving", 5, 1, 128, None, (1, 700), "bf16", "bf16", True, 256, seed=3),
+    W.Workload("ragged_mtp_fp8", 3, 2, 128, None, (2, 300), "bf16", "e4m3", True, 128, seed=4),
+    W.Workload("heads32", 2, 1, 32, None, (65, 129), "bf16", "bf16", True, 64, seed=5),
+    W.Workload("heads64_t2", 2, 2, 64, None, (190, 260), "bf16", "bf16", False, 128, seed=6),
+    W.Workload("f32_ragged", 3, 1, 16, None, (1, 333), "f32", "f32", True, 128, seed=7),
+    W.Workload("one_row", 2, 1, 128, 1, None, "bf16", "bf16", True, 64, seed=8),
+    W.Workload("all_new", 2, 2, 128, 2, None, "bf16", "e4m3", True, 64, seed=9),
+]
+
+
+def _check(dw: DeviceWorkload, seqs, naive=None, gain=None):
+    w = dw.w
+    out = dw.run()
+    torch.cuda.synchronize()
+    assert int(dw.step.err.item()) == 0
+    tol = TOL[w.cache_dtype]
+    worst = 0.0
+    for b in seqs:
+        ref_out, ref_olat, ref_lse = reference_sequence(w, b, gain)
+        got = gpu_rows(out, b, w.q_len)
+        err = oracle.normwise_rel_err(got, ref_out)
+        worst = max(worst, err)
+        assert err < tol, f"{w.name} seq {b}: out err {err:.3e} >= {tol}"
+        assert oracle.normwise_rel_err(gpu_rows(dw.step.o_lat, b, w.q_len), ref_olat) < tol
+        np.testing.assert_allclose(gpu_rows(dw.step.lse, b, w.q_len), ref_lse, atol=10 * tol)
+    if naive is not None:
+        b, heads = naive
+        ref, _, _ = reference_sequence(w, b, gain, heads=heads, form="naive")
+        got = gpu_rows(out, b, w.q_len)
+        got = got if heads is None else got[:, heads]
+        assert oracle.normwise_rel_err(got, ref) < tol, f"{w.name}: naive-form check"
+    return worst
+
+
+@pytest.mark.parametrize("name,seqs,naive", FULL, ids=[f[0] for f in FULL])
+def test_full_workload(name, seqs, naive):
+    dw = DeviceWorkload(W.WORKLOADS[name])
+    _check(dw, seqs, naive)
+
+
+@pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
+def test_small_workload_all_rows(w):
+    dw = DeviceWorkload(w)
+    _check(dw, range(w.batch), (0, None if w.n_heads <= 32 else [0, w.n_heads - 1]))
+
+
+def test_norm_gain_is_applied():
+    w = SMALL[0]
+    gain = W.norm_gain(w, "random")
+    dw = DeviceWorkload(w, norm_gain=gain)
+    _check(dw, range(w.batch), None, gain=gain)
+
+
+def test_repeated_steps_are_deterministic():
+    """Re-appending the same new rows and attending again gives identical bits."""
+    dw = DeviceWorkload(W.WORKLOADS["serving"])
+    a = dw.run().clone()
+    b = dw.run().clone()
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
