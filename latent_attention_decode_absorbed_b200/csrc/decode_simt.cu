@@ -53,7 +53,8 @@ __global__ void __launch_bounds__(512) decode_simt_kernel(DecodeArgs a) {
       float sc = 1.f;
       if (threadIdx.x < n) {
         const int j = j0 + threadIdx.x;
-        const int page = a.block_table[(size_t)b * a.max_pages + j / a.page_size];
+        const int pidx = j / a.page_size;
+        const int page = pidx < a.max_pages ? a.block_table[(size_t)b * a.max_pages + pidx] : -1;
         if (page >= 0 && page < a.num_pages) {
           sl = (long long)page * a.page_size + j % a.page_size;
           if (CK == MLA_E4M3) sc = a.cache_scale[sl];
