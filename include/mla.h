@@ -25,8 +25,8 @@
  * Conventions for every entry point
  *  - Pointers named as device pointers must be device memory (or managed
  *    memory) of the current device; the caller owns all memory.  No entry
- *    point allocates, frees or keeps device memory, except the tensor-map
- *    cache noted at mla_decode_fwd.
+ *    point allocates or frees device memory; the only device memory the
+ *    library itself holds is the fixed scratch array of mla_decode_static.
  *  - Tensors are dense, row-major, with the shapes given; device pointers must
  *    be 16-byte aligned (the cache 128-byte aligned).
  *  - Calls are asynchronous on `stream`; a return of MLA_OK means the work was
@@ -209,6 +209,45 @@ mla_status mla_combine(const float* o_part, const float* lse_part, int rows, int
  */
 mla_status mla_out_uv(const void* o_lat, const void* w_uv, void* out, int rows, int n_heads,
                       mla_dtype dtype, cudaStream_t stream);
+
+/*
+ * mla_decode_static
+ * Split-KV attention and its combine in one call that allocates nothing and
+ * takes no workspace: the same result as mla_decode_fwd followed by
+ * mla_combine, with the split partials kept in a scratch array that the
+ * library itself holds in device memory.  This call has no counterpart in
+ * the pages; it exists for callers that cannot allocate device memory on
+ * their own, e.g. a plugin whose host framework owns every device allocation,
+ * or a latency-critical serving loop where cudaMalloc's implicit device-wide
+ * synchronisation would stall the other streams.
+ *
+ *   Arguments as for mla_decode_fwd, except that the partials are internal:
+ *   o_lat   device [batch*q_len, n_heads, 512] of o_dtype (F32 or BF16)
+ *   lse_out device float [batch*q_len, n_heads] or NULL
+ *
+ * Limits and sharing:
+ *  - batch*q_len*n_heads*num_splits must not exceed MLA_STATIC_MAX_PARTIALS
+ *    (8192 partial rows, 16.8 MB of fp32 scratch); larger requests return
+ *    MLA_ERR_INVALID_ARG with the numbers in mla_last_error_message(), and
+ *    nothing is enqueued.  Use mla_decode_fwd + mla_combine for them.
+ *  - The scratch is a statically sized array in the library's device code:
+ *    every GPU that loads the library holds it until the process exits.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress, no allocation) with that device current; make
+ *    that first call before any stream capture begins.
+ *  - Every call uses the same array and it keeps the last call's contents.
+ *    Each call writes every partial it reads before reading it, so nothing
+ *    needs clearing.  Calls whose GPU work overlaps (on different streams,
+ *    or from different host threads without ordering) race on the array.
+ */
+#define MLA_STATIC_MAX_PARTIALS 8192
+mla_status mla_decode_static(const void* q_abs, mla_dtype q_dtype, const void* cache,
+                             const float* cache_scale, mla_dtype cache_dtype, int num_pages,
+                             const int32_t* block_table, int max_pages_per_seq, int page_size,
+                             const int32_t* seq_lens, int batch, int q_len, int n_heads,
+                             int num_splits, int split_tokens, float softmax_scale,
+                             void* o_lat, mla_dtype o_dtype, float* lse_out, int32_t* err_word,
+                             cudaStream_t stream);
 
 #ifdef __cplusplus
 }

@@ -31,6 +31,7 @@ _SIGS = {
     "mla_decode_fwd": ("i", "pippiipiipiiiiifpppp"),
     "mla_combine": ("i", "ppiiipipp"),
     "mla_out_uv": ("i", "pppiiip"),
+    "mla_decode_static": ("i", "pippiipiipiiiiifpippp"),
 }
 _CT = {"p": ctypes.c_void_p, "i": ctypes.c_int, "f": ctypes.c_float, "d": ctypes.c_double,
        "s": ctypes.c_char_p}
@@ -138,5 +139,19 @@ def mla_out_uv(o_lat, w_uv, out, rows, n_heads, dtype, stream=None):
     _check("mla_out_uv", lib().mla_out_uv(_ptr(o_lat), _ptr(w_uv), _ptr(out), int(rows), int(n_heads),
                                           int(dtype), _stream(stream)))
 
+
+def mla_decode_static(q_abs, q_dtype, cache, cache_scale, cache_dtype, num_pages, block_table,
+                      max_pages_per_seq, page_size, seq_lens, batch, q_len, n_heads, num_splits,
+                      split_tokens, softmax_scale, o_lat, o_dtype, lse_out=None, err_word=None, stream=None):
+    """Attention + combine without caller workspace (library-held scratch);
+    see the header for its size limit and sharing rules."""
+    _check("mla_decode_static", lib().mla_decode_static(
+        _ptr(q_abs), int(q_dtype), _ptr(cache), _ptr(cache_scale), int(cache_dtype), int(num_pages),
+        _ptr(block_table), int(max_pages_per_seq), int(page_size), _ptr(seq_lens), int(batch),
+        int(q_len), int(n_heads), int(num_splits), int(split_tokens), float(softmax_scale),
+        _ptr(o_lat), int(o_dtype), _ptr(lse_out), _ptr(err_word), _stream(stream)))
+
+
+MLA_STATIC_MAX_PARTIALS = 8192
 
 from .step import DecodeStep  # noqa: E402,F401
