@@ -172,9 +172,13 @@ mla_status mla_absorb_q(const void* q_nope, const void* q_pe, const void* w_uk, 
  *   lse_part    device float [batch*q_len, n_heads, num_splits]
  *   err_word    device int32 or NULL (MLA_DEVERR_PAGE, MLA_DEVERR_TIMEOUT)
  * Supported: page_size 64; q_dtype F32 with cache F32; q_dtype BF16 with cache
- * BF16 or E4M3.  BF16/E4M3 run on the tcgen05 tensor cores (bf16 operands,
- * fp32 accumulation); F32 runs exact fp32 on the CUDA cores.  The library
- * caches TMA descriptors per (cache pointer, pool size) on the host.
+ * BF16 or E4M3.  BF16 runs on the tcgen05 tensor cores (bf16 operands, fp32
+ * accumulation, one CTA pair per (query row, split)); F32 runs exact fp32 on
+ * the CUDA cores.
+ * Pool contract: the tensor-core path reads whole 64-row pages.  Rows of a
+ * sequence's last page beyond its length, and page 0 (read in place of a
+ * block-table entry outside the pool), enter the contraction with zero
+ * weight, so they must hold finite values: allocate the pool zero-filled.
  */
 mla_status mla_decode_fwd(const void* q_abs, mla_dtype q_dtype, const void* cache,
                           const float* cache_scale, mla_dtype cache_dtype, int num_pages,

@@ -1,0 +1,620 @@
+// Split-KV latent attention on the tcgen05 tensor cores (bf16 operands,
+// fp32 accumulation), one CTA pair per (query row, split).
+//
+// What it computes ("DeepSeek-V2: MLA Explained", "MLA Full Formulas" part 3
+// with the absorption of "Optimization Note"): for each head h of query row
+// r and each cached row j of the split that the query sees,
+//   z_j = scale * (q_abs[r,h,0:512] . c_j + q_abs[r,h,512:576] . k_j)
+// then the split's normalised softmax-weighted mean of the latents c_j and
+// its log-normaliser.
+//
+// How.  All heads share the cached rows, so the two contractions are dense
+// GEMMs per tile of 256 rows, computed transposed so that neither the
+// [heads x 576] query nor the [heads x 512] fp32 accumulator has to fit one
+// SM:
+//   S^T[256 rows x H]  = K[256 x 576] . Q[H x 576]^T        (cta_group::2, M=256)
+//   O^T[512 dims x H] += V^T[512 x 256] . P^T[H x 256]^T    (two M=256 MMAs)
+// CTA r of the pair holds rows [128r, 128r+128) of each tile for S^T, half of
+// the heads of Q and of P^T (the split B operand), and dims
+// {[128r,128r+128), [256+128r, 256+128r+128)} of O^T in its TMEM.  TMEM per
+// CTA: two S^T buffers (2 x 128 columns) + O^T (2 x 128 columns) = 512.
+//
+// Cache rows stream through a ring of 16 KB shared-memory slots filled by TMA
+// (one 64-row page x 64 columns per 8 KB box, 128-byte swizzle).  The same
+// bytes serve as the K-major A operand of S^T (rows x dims) and the MN-major
+// A operand of O^T (dims x rows).  Warp roles per CTA: 0 TMA producer and
+// TMEM allocator, 1 MMA issuer (leader CTA only), 2-9 softmax (two
+// warpgroups, one per half of the heads; thread = cached row).
+//
+// Softmax per tile: each warp takes the per-head max of its 32 rows with
+// redux.sync, the 4 warps of a warpgroup combine through shared memory, the
+// pair exchanges its maxima through distributed shared memory, and the
+// running max only moves when the tile max exceeds it by more than 2^8 (the
+// accumulator is rescaled in TMEM then).  P = 2^(u - m) is written as bf16
+// straight into the P^T operand of the CTA that owns those heads.
+#include <math.h>
+
+#include "mla_device.cuh"
+#include "mla_internal.h"
+#include "sm100.cuh"
+
+namespace mla {
+namespace {
+
+using namespace sm100;
+
+constexpr int kThreads = 320;
+constexpr int kSlotBytes = 16384;
+constexpr int kBoxBytes = 8192;           // 64 rows x 128 bytes
+constexpr int kTile = 256;                // cached rows per pair tile
+constexpr int kChunks = 9;                // 576 / 64 column chunks
+constexpr float kRescaleLog2 = 8.0f;      // lazy rescale threshold (log2 units)
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
+
+struct TcParams {
+  int n_heads, q_len, batch;
+  const int32_t* block_table;
+  int max_pages, num_pages;
+  const int32_t* seq_lens;
+  int num_splits, split_tokens;
+  float scale_log2;            // softmax_scale * log2(e)
+  float* o_part;
+  float* lse_part;
+  int32_t* err;
+};
+
+template <int NH>
+struct Layout {
+  static constexpr int HPW = NH / 2;                      // heads per CTA / per warpgroup
+  static constexpr int kRingSlots = 7;
+  static constexpr int kQChunk = HPW * 128;               // one 64-column chunk of this CTA's Q rows
+  static constexpr int kPChunk = HPW * 128;               // 64 rows of P^T for this CTA's heads
+  static constexpr int kRing = 0;
+  static constexpr int kQ = kRing + kRingSlots * kSlotBytes;
+  static constexpr int kP = kQ + kChunks * kQChunk;
+  static constexpr int kMisc = kP + 4 * kPChunk;
+  // misc area (bytes from kMisc)
+  static constexpr int kBars = 0;                          // 64 barriers max
+  static constexpr int kTmemSlot = 64 * 8;
+  static constexpr int kAbort = kTmemSlot + 4;      // +8, +12: per-warpgroup flags
+  static constexpr int kMused = kTmemSlot + 32;            // float [2][NH]
+  static constexpr int kRed = kMused + 2 * NH * 4;          // float [2 wg][4 warps][HPW]
+  static constexpr int kOwnMax = kRed + 2 * 4 * HPW * 4;    // float [NH]
+  static constexpr int kXMax = kOwnMax + NH * 4;            // float [2][NH]   written by the peer
+  static constexpr int kLOwn = kXMax + 2 * NH * 4;          // float [NH]
+  static constexpr int kLX = kLOwn + NH * 4;                // float [NH]      written by the peer
+  static constexpr int kMiscBytes = kLX + NH * 4;
+  static constexpr int kSmem = kMisc + kMiscBytes + 1024;  // + alignment slack
+};
+
+// barrier indices in the misc area
+template <int NS>
+struct Bars {
+  static constexpr int full = 0;               // [NS]  leader: TMA bytes of both CTAs
+  static constexpr int empty = NS;             // [NS]  both: MMA done with the slot
+  static constexpr int s_full = 2 * NS;        // [2]   both: S^T buffer ready
+  static constexpr int s_free = 2 * NS + 2;    // [2]   leader: both CTAs read the S^T buffer
+  static constexpr int p_full = 2 * NS + 4;    //       leader: both CTAs wrote P^T
+  static constexpr int o_done = 2 * NS + 5;    //       both: O^T MMAs of the tile done
+  static constexpr int mx_full = 2 * NS + 6;   // [2]   both: the peer's tile maxima arrived
+  static constexpr int q_full = 2 * NS + 8;    //       leader: Q of both CTAs loaded
+  static constexpr int l_full = 2 * NS + 9;    //       both: the peer's row sums arrived
+};
+
+__device__ __forceinline__ float redux_max(float v) {
+  float r;
+  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+  return r;
+}
+
+// Sum over the 32 lanes of a warp of each of C per-lane values, returned
+// transposed: lane l gets the sum of index l % C.  log2(32) shuffle stages;
+// the split stages halve the values each lane carries, so C = 32 costs 31
+// shuffles instead of the 160 of C independent reductions.  v is clobbered.
+template <int C>
+__device__ __forceinline__ float transpose_reduce(float* v, int lane) {
+#pragma unroll
+  for (int off = 16; off >= C; off >>= 1) {
+#pragma unroll
+    for (int j = 0; j < C; ++j) v[j] += __shfl_xor_sync(0xffffffffu, v[j], off);
+  }
+#pragma unroll
+  for (int off = C / 2; off >= 1; off >>= 1) {
+    const bool up = (lane & off) != 0;
+#pragma unroll
+    for (int j = 0; j < off; ++j) {
+      const float keep = up ? v[j + off] : v[j];
+      const float send = up ? v[j] : v[j + off];
+      v[j] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+  }
+  return v[0];
+}
+
+__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+__device__ __forceinline__ void st_cluster_b32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+// page id of a cached row of sequence b (0 for rows outside the table or the
+// pool: those rows are masked by the softmax, and page 0 is readable memory)
+__device__ __forceinline__ int page_of(const TcParams& p, int b, int row, bool* ok) {
+  const int pidx = row >> 6;
+  int pg = -1;
+  if (pidx < p.max_pages) pg = p.block_table[(size_t)b * p.max_pages + pidx];
+  *ok = pg >= 0 && pg < p.num_pages;
+  return *ok ? pg : 0;
+}
+
+template <int NH>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_constant__ CUtensorMap tm_q,
+                     const TcParams p) {
+  using LY = Layout<NH>;
+  constexpr int HPW = LY::HPW;
+  constexpr int NS = LY::kRingSlots;
+  using B = Bars<NS>;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t s_base = smem_u32(smem);
+  const uint32_t s_ring = s_base + LY::kRing, s_q = s_base + LY::kQ, s_p = s_base + LY::kP;
+  uint8_t* misc = smem + LY::kMisc;
+  const uint32_t s_misc = s_base + LY::kMisc;
+  auto bar = [&](int i) -> uint32_t { return s_misc + LY::kBars + 8 * i; };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + LY::kAbort);
+  float* m_used = reinterpret_cast<float*>(misc + LY::kMused);
+  float* red = reinterpret_cast<float*>(misc + LY::kRed);
+  float* own_max = reinterpret_cast<float*>(misc + LY::kOwnMax);
+  float* x_max = reinterpret_cast<float*>(misc + LY::kXMax);
+  float* l_own = reinterpret_cast<float*>(misc + LY::kLOwn);
+  float* l_x = reinterpret_cast<float*>(misc + LY::kLX);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const uint32_t peer = rank ^ 1u;
+  const bool leader = rank == 0;
+
+  // ---- unit: (query row r, split s)
+  const int unit = blockIdx.x >> 1;
+  const int S = p.num_splits;
+  const int r = unit / S, s = unit % S;
+  const int b = r / p.q_len, t = r % p.q_len;
+  const int L = p.seq_lens[b];
+  const int n_vis = L - p.q_len + t + 1;
+  const int lo = s * p.split_tokens;
+  const int hi = min(lo + p.split_tokens, n_vis);
+  const int n_tok = hi - lo;
+  const int n_tiles = n_tok > 0 ? (n_tok + kTile - 1) / kTile : 0;
+
+  // ---- set-up: barriers, TMEM, cluster sync
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(bar(B::full + i), 1);
+      mbar_init(bar(B::empty + i), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(B::s_full + i), 1);
+      mbar_init(bar(B::s_free + i), 16);
+      mbar_init(bar(B::mx_full + i), 2);
+    }
+    mbar_init(bar(B::p_full), 16);
+    mbar_init(bar(B::o_done), 1);
+    mbar_init(bar(B::q_full), 1);
+    mbar_init(bar(B::l_full), 2);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  for (int i = threadIdx.x; i < 2 * NH; i += kThreads) m_used[i] = -INFINITY;
+  if (warp == 0) tmem_alloc_pair(s_misc + LY::kTmemSlot, kTmemCols);
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(misc + LY::kTmemSlot);
+
+  if (n_tiles == 0) {
+    // nothing visible in this split: o = 0, lse = -inf (heads split by rank)
+    for (int i = threadIdx.x; i < p.n_heads * MLA_D_C; i += kThreads) {
+      const int h = i / MLA_D_C, d = i % MLA_D_C;
+      if ((h & 1) != (int)rank) continue;
+      p.o_part[(((size_t)r * p.n_heads + h) * S + s) * MLA_D_C + d] = 0.f;
+      if (d == 0) p.lse_part[((size_t)r * p.n_heads + h) * S + s] = -INFINITY;
+    }
+  } else if (warp == 0) {
+    // ================= TMA producer (both CTAs) =================
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_cache);
+      tma_prefetch_desc(&tm_q);
+      const uint32_t q_bar = mapa(bar(B::q_full), 0);
+      if (leader) mbar_arrive_expect_tx(bar(B::q_full), 2u * kChunks * LY::kQChunk);
+      for (int c = 0; c < kChunks; ++c)
+        tma_load_3d_pair(s_q + c * LY::kQChunk, &tm_q, 64 * c, (int)rank * HPW, r, q_bar);
+      uint32_t kc = 0;
+      bool ok = true;
+      auto take_slot = [&](uint32_t& slot) -> bool {
+        slot = kc % NS;
+        const uint32_t ph = (kc / NS) & 1u;
+        if (!mbar_wait(bar(B::empty + slot), ph ^ 1u, abort_flag)) return false;
+        if (leader) mbar_arrive_expect_tx(bar(B::full + slot), 2u * kSlotBytes);
+        ++kc;
+        return true;
+      };
+      auto emit_o = [&](int j) -> bool {
+        for (int pg_i = 0; pg_i < 4; ++pg_i) {
+          const int row0 = lo + kTile * j + 64 * pg_i;
+          if (row0 >= hi) break;
+          bool vld;
+          const int pg = page_of(p, b, row0, &vld);
+          for (int bb = 0; bb < 2; ++bb) {
+            uint32_t slot;
+            if (!take_slot(slot)) return false;
+            const uint32_t dst = s_ring + slot * kSlotBytes;
+            const uint32_t fb = mapa(bar(B::full + slot), 0);
+            const int x0 = 256 * bb + 128 * (int)rank;
+            tma_load_2d_pair(dst, &tm_cache, x0, pg * 64, fb);
+            tma_load_2d_pair(dst + kBoxBytes, &tm_cache, x0 + 64, pg * 64, fb);
+          }
+        }
+        return true;
+      };
+      for (int i = 0; i < n_tiles && ok; ++i) {
+        const int row0 = lo + kTile * i + 128 * (int)rank;
+        bool v0, v1;
+        const int pg0 = page_of(p, b, row0, &v0);
+        const int pg1 = page_of(p, b, row0 + 64, &v1);
+        for (int c = 0; c < kChunks && ok; ++c) {
+          uint32_t slot;
+          if (!take_slot(slot)) { ok = false; break; }
+          const uint32_t dst = s_ring + slot * kSlotBytes;
+          const uint32_t fb = mapa(bar(B::full + slot), 0);
+          tma_load_2d_pair(dst, &tm_cache, 64 * c, pg0 * 64, fb);
+          tma_load_2d_pair(dst + kBoxBytes, &tm_cache, 64 * c, pg1 * 64, fb);
+        }
+        if (ok && i >= 1) ok = emit_o(i - 1);
+      }
+      if (ok) emit_o(n_tiles - 1);
+    }
+  } else if (warp == 1) {
+    // ================= MMA issuer (leader CTA) =================
+    if (leader && lane == 0) {
+      constexpr uint32_t idS = idesc_f16(256, NH, false, false);
+      constexpr uint32_t idO = idesc_f16(256, NH, true, false);
+      uint32_t kc = 0;
+      bool ok = mbar_wait(bar(B::q_full), 0, abort_flag);
+      tc_fence_after();
+      auto wait_slot = [&](uint32_t& slot) -> bool {
+        slot = kc % NS;
+        const uint32_t ph = (kc / NS) & 1u;
+        if (!mbar_wait(bar(B::full + slot), ph, abort_flag)) return false;
+        tc_fence_after();
+        ++kc;
+        return true;
+      };
+      auto issue_o = [&](int j) -> bool {
+        if (!mbar_wait(bar(B::p_full), j & 1, abort_flag)) return false;
+        tc_fence_after();
+        for (int pg_i = 0; pg_i < 4; ++pg_i) {
+          if (lo + kTile * j + 64 * pg_i >= hi) break;
+          for (int bb = 0; bb < 2; ++bb) {
+            uint32_t slot;
+            if (!wait_slot(slot)) return false;
+            const uint32_t a0 = s_ring + slot * kSlotBytes;
+            for (int ks = 0; ks < 4; ++ks) {
+              const uint64_t ad = smem_desc_sw128(a0 + ks * 2048, kBoxBytes, 1024);
+              const uint64_t bd = smem_desc_sw128(s_p + pg_i * LY::kPChunk + ks * 32, 16, 1024);
+              mma_pair_f16(tmem + kColO + bb * 128, ad, bd, idO, (j | pg_i | ks) != 0);
+            }
+            mma_commit_pair(bar(B::empty + slot), 0x3);
+          }
+        }
+        mma_commit_pair(bar(B::o_done), 0x3);
+        return true;
+      };
+      for (int i = 0; i < n_tiles && ok; ++i) {
+        const int sb = i & 1;
+        if (i >= 2) {
+          if (!mbar_wait(bar(B::s_free + sb), ((i - 2) >> 1) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+        }
+        const uint32_t d = tmem + (sb ? kColS1 : kColS0);
+        for (int c = 0; c < kChunks; ++c) {
+          uint32_t slot;
+          if (!wait_slot(slot)) { ok = false; break; }
+          const uint32_t a0 = s_ring + slot * kSlotBytes;
+          for (int ks = 0; ks < 4; ++ks) {
+            const uint64_t ad = smem_desc_sw128(a0 + ks * 32, 16, 1024);
+            const uint64_t bd = smem_desc_sw128(s_q + c * LY::kQChunk + ks * 32, 16, 1024);
+            mma_pair_f16(d, ad, bd, idS, (c | ks) != 0);
+          }
+          mma_commit_pair(bar(B::empty + slot), 0x3);
+        }
+        if (!ok) break;
+        mma_commit_pair(bar(B::s_full + sb), 0x3);
+        if (i >= 1) ok = issue_o(i - 1);
+      }
+      if (ok) issue_o(n_tiles - 1);
+    }
+  } else if (warp >= 2) {
+    // ================= softmax (both CTAs, 8 warps) =================
+    // Per tile, in column chunks of C heads so that few registers are live:
+    //   A  tile max per head (redux over a warp's rows, then over 4 warps)
+    //   -- warp 0 of the group exchanges maxima with the peer and sets the
+    //      new running max (and the rescale factors) in shared memory
+    //   B  P = 2^(u - m) written to P^T, running row sums updated
+    constexpr int C = HPW < 32 ? HPW : 32;
+    const int g = (warp - 2) >> 2;             // warpgroup: heads [g*HPW, (g+1)*HPW)
+    const int q = warp & 3;                    // TMEM lane quadrant
+    const int tok = 32 * q + lane;             // row within this CTA's half of the tile
+    const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
+    const uint32_t p_dst = (g == (int)rank) ? s_p : mapa(s_p, (uint32_t)g);
+    const bool p_remote = g != (int)rank;
+    float* red_g = red + g * 4 * HPW;
+    float* alpha = own_max;                    // reused after the tile max is consumed
+    volatile int* changed_flag = reinterpret_cast<volatile int*>(misc + LY::kTmemSlot + 8) + g;
+    // running row sums of this warp's 32 rows: chunk k, head C*k + lane % C
+    float l_acc[HPW / C];
+#pragma unroll
+    for (int k = 0; k < HPW / C; ++k) l_acc[k] = 0.f;
+    bool ok = true;
+    for (int i = 0; i < n_tiles; ++i) {
+      const int sb = i & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(B::s_full + sb), (i >> 1) & 1, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t sc = tmem + lane_addr + (sb ? kColS1 : kColS0) + g * HPW;
+      const int row = lo + kTile * i + 128 * (int)rank + tok;
+      bool vld = row < hi;
+      if (vld) {
+        bool pok;
+        (void)page_of(p, b, row, &pok);
+        if (!pok) { vld = false; flag_error(p.err, MLA_DEVERR_PAGE); }
+      }
+      const float sl = vld ? p.scale_log2 : 0.f;
+      // ---- A: per-head tile max
+#pragma unroll
+      for (int k = 0; k < HPW / C; ++k) {
+        float u[C];
+        tmem_ld<C>(sc + C * k, u);
+        tmem_wait_ld();
+#pragma unroll
+        for (int h = 0; h < C; ++h) {
+          const float mx = redux_max(vld ? u[h] * sl : -INFINITY);
+          if (lane == (h & 31)) red_g[q * HPW + C * k + h] = mx;
+        }
+      }
+      named_barrier(1 + g, 128);
+      const int xb = i & 1;
+      const float* m_prev = m_used + ((i + 1) & 1) * NH + g * HPW;
+      float* m_next = m_used + (i & 1) * NH + g * HPW;
+      if (q == 0) {
+        for (int h = lane; h < HPW; h += 32) {
+          const float tm = fmaxf(fmaxf(red_g[h], red_g[HPW + h]), fmaxf(red_g[2 * HPW + h], red_g[3 * HPW + h]));
+          own_max[g * HPW + h] = tm;
+          st_cluster_f32(mapa(smem_u32(x_max + xb * NH + g * HPW + h), peer), tm);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(mapa(bar(B::mx_full + xb), peer));
+        if (__all_sync(0xffffffffu, mbar_wait(bar(B::mx_full + xb), (i >> 1) & 1, abort_flag))) {
+          int ch = 0;
+          for (int h = lane; h < HPW; h += 32) {
+            const float mt = fmaxf(own_max[g * HPW + h], x_max[xb * NH + g * HPW + h]);
+            const float mo = m_prev[h];
+            const float mn = (mt > mo + kRescaleLog2) ? mt : mo;
+            m_next[h] = mn;
+            // rescale factor for sums and accumulator kept so far (0 when nothing was kept)
+            alpha[g * HPW + h] = (mo == -INFINITY) ? 0.f : exp2f(mo - mn);
+            ch |= (mn != mo);
+          }
+          ch = __any_sync(0xffffffffu, ch);
+          if (lane == 0) *changed_flag = ch;
+        }
+      }
+      named_barrier(1 + g, 128);
+      if (*abort_flag) { ok = false; break; }
+      const bool changed = *changed_flag != 0;
+      // the previous tile's O^T MMAs must be done: P^T buffer reuse and rescale
+      if (i >= 1) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(B::o_done), (i - 1) & 1, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+        if (changed) {
+#pragma unroll
+          for (int bb = 0; bb < 2; ++bb) {
+#pragma unroll
+            for (int k = 0; k < HPW / C; ++k) {
+              const uint32_t oc = tmem + lane_addr + kColO + bb * 128 + g * HPW + C * k;
+              float o[C];
+              tmem_ld<C>(oc, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int h = 0; h < C; ++h) o[h] *= alpha[g * HPW + C * k + h];
+              tmem_st<C>(oc, o);
+            }
+          }
+          tmem_wait_st();
+        }
+      }
+      // ---- B: probabilities, row sums, P^T (bf16, pairs of rows per 32-bit store)
+      const int kt = 128 * (int)rank + tok;
+      const int ke = kt & ~1;
+      const int w = ke & 63;
+      const uint32_t row_base = (ke >> 6) * LY::kPChunk + (w & 7) * 2;
+#pragma unroll
+      for (int k = 0; k < HPW / C; ++k) {
+        float u[C];
+        tmem_ld<C>(sc + C * k, u);
+        tmem_wait_ld();
+#pragma unroll
+        for (int h = 0; h < C; ++h) {
+          const float mn = m_next[C * k + h];
+          u[h] = vld ? exp2f(u[h] * sl - (mn == -INFINITY ? 0.f : mn)) : 0.f;
+        }
+#pragma unroll
+        for (int h = 0; h < C; h += 2) {
+          const float send = (lane & 1) ? u[h] : u[h + 1];
+          const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
+          const int hr = C * k + ((lane & 1) ? h + 1 : h);
+          __nv_bfloat162 pk = (lane & 1) ? __floats2bfloat162_rn(recv, u[h + 1]) : __floats2bfloat162_rn(u[h], recv);
+          const uint32_t val = *reinterpret_cast<uint32_t*>(&pk);
+          const uint32_t off = row_base + hr * 128 + ((((w >> 3) ^ (hr & 7))) << 4);
+          if (p_remote) st_cluster_b32(p_dst + off, val);
+          else asm volatile("st.shared.b32 [%0], %1;" ::"r"(p_dst + off), "r"(val) : "memory");
+        }
+        const float ls = transpose_reduce<C>(u, lane);
+        l_acc[k] = changed ? fmaf(l_acc[k], alpha[g * HPW + C * k + (lane % C)], ls) : l_acc[k] + ls;
+      }
+      tc_fence_before();
+      fence_proxy_async_cluster();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive_cluster(mapa(bar(B::s_free + sb), 0));
+        mbar_arrive_cluster(mapa(bar(B::p_full), 0));
+      }
+    }
+    // ---- epilogue: normalise O^T by the row sums, write o_part and lse
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(B::o_done), (n_tiles - 1) & 1, abort_flag));
+    if (ok) {
+      tc_fence_after();
+#pragma unroll
+      for (int k = 0; k < HPW / C; ++k)
+        if (lane < C) red_g[q * HPW + C * k + lane] = l_acc[k];
+      named_barrier(1 + g, 128);
+      float* inv_l = own_max;
+      if (q == 0) {
+        for (int h = lane; h < HPW; h += 32) {
+          const float lt = red_g[h] + red_g[HPW + h] + red_g[2 * HPW + h] + red_g[3 * HPW + h];
+          l_own[g * HPW + h] = lt;
+          st_cluster_f32(mapa(smem_u32(l_x + g * HPW + h), peer), lt);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(mapa(bar(B::l_full), peer));
+        if (__all_sync(0xffffffffu, mbar_wait(bar(B::l_full), 0, abort_flag))) {
+          const float* m_fin = m_used + ((n_tiles - 1) & 1) * NH + g * HPW;
+          for (int h = lane; h < HPW; h += 32) {
+            const int hg = g * HPW + h;
+            const float lt = l_own[hg] + l_x[hg];
+            inv_l[hg] = lt > 0.f ? 1.0f / lt : 0.f;
+            if (leader && hg < p.n_heads)
+              p.lse_part[((size_t)r * p.n_heads + hg) * S + s] =
+                  lt > 0.f ? (m_fin[h] + log2f(lt)) * 0.69314718055994531f : -INFINITY;
+          }
+        }
+      }
+      named_barrier(1 + g, 128);
+      if (!*abort_flag) {
+        const size_t hstride = (size_t)S * MLA_D_C;
+#pragma unroll 1
+        for (int bb = 0; bb < 2; ++bb) {
+          const int d = 256 * bb + 128 * (int)rank + tok;
+#pragma unroll 1
+          for (int k = 0; k < HPW / C; ++k) {
+            const int h0 = g * HPW + C * k;
+            float* op = p.o_part + ((size_t)r * p.n_heads * S + s) * MLA_D_C + d + (size_t)h0 * hstride;
+            float o[C];
+            tmem_ld<C>(tmem + lane_addr + kColO + bb * 128 + h0, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int h = 0; h < C; ++h) {
+              if (h0 + h < p.n_heads) *op = o[h] * inv_l[h0 + h];
+              op += hstride;
+            }
+          }
+        }
+      }
+    }
+  }
+
+  // ---- teardown
+  if (*abort_flag) {
+    if (threadIdx.x == 0) flag_error(p.err, MLA_DEVERR_TIMEOUT);
+    // let copies and MMAs already in flight land before the memory is released
+    const uint64_t t0 = globaltimer();
+    while (globaltimer() - t0 < 2000000ull) {
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  }
+  return fn;
+}
+
+template <int NH>
+cudaError_t launch_nh(const DecodeArgs& a, const CUtensorMap& tc, const CUtensorMap& tq, cudaStream_t st) {
+  using LY = Layout<NH>;
+  cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<NH>, cudaFuncAttributeMaxDynamicSharedMemorySize, LY::kSmem);
+  if (e != cudaSuccess) return e;
+  TcParams p{a.n_heads, a.q_len, a.batch, a.block_table, a.max_pages, a.num_pages, a.seq_lens, a.num_splits,
+             a.split_tokens, a.softmax_scale * 1.4426950408889634f, a.o_part, a.lse_part, a.err};
+  const long long units = (long long)a.batch * a.q_len * a.num_splits;
+  dim3 grid((unsigned)(2 * units));
+  decode_tc_kernel<NH><<<grid, kThreads, LY::kSmem, st>>>(tc, tq, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool decode_tc_supported(const DecodeArgs& a) {
+  return a.q_dtype == MLA_BF16 && a.cache_dtype == MLA_BF16 && a.page_size == 64 &&
+         (long long)a.batch * a.q_len * a.num_splits * 2 < (1ll << 31);
+}
+
+cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  const int NH = a.n_heads <= 16 ? 16 : a.n_heads <= 32 ? 32 : a.n_heads <= 64 ? 64 : 128;
+  const int HPW = NH / 2;
+  CUtensorMap tc, tq;
+  {
+    cuuint64_t dims[2] = {MLA_D_ROW, (cuuint64_t)a.num_pages * 64};
+    cuuint64_t strides[1] = {MLA_D_ROW * 2};
+    cuuint32_t box[2] = {64, 64};
+    cuuint32_t es[2] = {1, 1};
+    if (enc(&tc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a.cache), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  {
+    cuuint64_t dims[3] = {MLA_D_ROW, (cuuint64_t)a.n_heads, (cuuint64_t)a.batch * a.q_len};
+    cuuint64_t strides[2] = {MLA_D_ROW * 2, (cuuint64_t)a.n_heads * MLA_D_ROW * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)HPW, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    if (enc(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(a.q_abs), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  switch (NH) {
+    case 16: return launch_nh<16>(a, tc, tq, st);
+    case 32: return launch_nh<32>(a, tc, tq, st);
+    case 64: return launch_nh<64>(a, tc, tq, st);
+    default: return launch_nh<128>(a, tc, tq, st);
+  }
+}
+
+}  // namespace mla

@@ -38,6 +38,9 @@ struct DecodeArgs {
   float* o_part; float* lse_part; int32_t* err;
 };
 cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t st);
+// tcgen05 path: bf16 queries over a bf16 cache
+bool decode_tc_supported(const DecodeArgs& a);
+cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st);
 
 cudaError_t launch_combine(const float* o_part, const float* lse_part, int rows, int n_heads,
                            int num_splits, void* o_lat, int o_dtype, float* lse_out,

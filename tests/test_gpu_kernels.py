@@ -203,6 +203,8 @@ CASES = [
     ("mtp_bf16", "bf16", [2, 190, 513], 2, 128, 128),
     ("heads16_bf16", "bf16", [333, 64], 1, 16, 128),
     ("heads64_mtp_bf16", "bf16", [260], 2, 64, 128),
+    ("heads48_bf16", "bf16", [200, 513], 1, 48, 256),
+    ("long_split_bf16", "bf16", [5000], 1, 128, 4096),
     ("ragged_e4m3", "e4m3", [5, 400, 1025], 2, 128, 256),
     ("tiny_f32", "f32", [256, 37], 1, 16, 64),
 ]
