@@ -12,8 +12,14 @@
  * The cache ("KV Compression - DeepSeek-V3", section "How it works") holds one
  * row of 576 numbers per token: the RMSNorm'd 512-wide joint KV latent c_kv
  * followed by the 64-wide RoPE'd key k_pe shared by all heads.  Rows live in
- * pages of `page_size` tokens; a per-sequence block table maps a sequence's
- * page slot to a page of one pool.
+ * pages of `page_size` = 64 tokens; a per-sequence block table maps a
+ * sequence's page slot to a page of one pool.
+ *
+ * Pool layout (page-blocked): cache[num_pages][9][64][64] - each page is nine
+ * contiguous blocks of [64 rows x 64 columns], block c holding columns
+ * 64c..64c+63 of the page's 64 rows.  Element (slot = page*64 + row, column d)
+ * sits at index ((page*9 + d/64)*64 + row)*64 + d%64.  Every tensor-core load
+ * of the decode is then one contiguous 8 or 16 KB read.
  *
  * A decode step for B sequences with T new tokens each, H heads:
  *   mla_cache_append  new kv_a rows -> cache rows (RMSNorm, RoPE, cast/quantise)
@@ -110,9 +116,9 @@ mla_status mla_rope_table(double theta, int max_pos, float* cos_out, float* sin_
  *   c   = kv_a[n, 0:512],  cache_c = c / sqrt(mean(c^2) + eps) * norm_gain
  *   k   = kv_a[n, 512:576], cache_k[2i] = k[2i] cos - k[2i+1] sin,
  *                           cache_k[2i+1] = k[2i] sin + k[2i+1] cos  (table row positions[n])
- *   row = [cache_c ; cache_k] stored at
- *         cache[(block_table[seq_ids[n], positions[n] / page_size] * page_size
- *                + positions[n] % page_size) * 576 ...]
+ *   row = [cache_c ; cache_k] stored at slot
+ *         block_table[seq_ids[n], positions[n] / page_size] * page_size + positions[n] % page_size
+ *         of the page-blocked pool (see the layout above)
  *   E4M3 cache: a = max|row|, cache_scale[slot] = a / 448,
  *         codes = e4m3_rne_satfinite(row * (448 / a)); a = 0 stores zeros and scale 0.
  * Arithmetic is fp32.
@@ -123,7 +129,7 @@ mla_status mla_rope_table(double theta, int max_pos, float* cos_out, float* sin_
  *   norm_gain   device float [512] or NULL (gain 1)
  *   eps         RMSNorm epsilon (>= 0)
  *   rope_cos, rope_sin device float [rope_max_pos, 32] (see mla_rope_table)
- *   cache       device [num_pages, page_size, 576] of cache_dtype (F32, BF16, E4M3)
+ *   cache       device [num_pages, 9, 64, 64] of cache_dtype (F32, BF16, E4M3), page-blocked
  *   cache_scale device float [num_pages, page_size] for E4M3, else ignored (may be NULL)
  *   err_word    device int32 or NULL; rows whose sequence, position or page is out of
  *               range are skipped and flagged (MLA_DEVERR_POSITION / MLA_DEVERR_PAGE)
@@ -163,7 +169,7 @@ mla_status mla_absorb_q(const void* q_nope, const void* q_pe, const void* w_uk, 
  *   o_part[r,h,s,:] = sum_j e^{z_j - m} c_j / sum_j e^{z_j - m}   over the split's visible j
  *   lse_part[r,h,s] = m + ln sum_j e^{z_j - m}  (natural log; -inf and o = 0 for an empty split)
  *   q_abs       device [batch*q_len, n_heads, 576], q_dtype F32 or BF16
- *   cache       device [num_pages, page_size, 576]; cache_scale as for mla_cache_append
+ *   cache       device [num_pages, 9, 64, 64], page-blocked; cache_scale as for mla_cache_append
  *   block_table device int32 [batch, max_pages_per_seq]
  *   seq_lens    device int32 [batch], q_len <= L_b <= max_pages_per_seq*page_size
  *   num_splits * split_tokens must cover the longest sequence; split_tokens is

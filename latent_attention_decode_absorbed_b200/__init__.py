@@ -93,6 +93,20 @@ def dtype_code(t) -> int:
             torch.float8_e4m3fn: MLA_E4M3}[t.dtype]
 
 
+def pack_cache_rows(rows):
+    """Logical cache rows [num_pages*64, 576] -> the page-blocked pool layout
+    [num_pages, 9, 64, 64] (nine [64 rows x 64 columns] blocks per page).
+    A pure layout transform (torch tensors, any dtype)."""
+    n = rows.shape[0] // PAGE
+    return rows.reshape(n, PAGE, D_ROW // 64, 64).permute(0, 2, 1, 3).contiguous()
+
+
+def unpack_cache_rows(cache):
+    """Page-blocked pool [num_pages, 9, 64, 64] -> logical rows [num_pages*64, 576]."""
+    n = cache.shape[0]
+    return cache.reshape(n, D_ROW // 64, PAGE, 64).permute(0, 2, 1, 3).reshape(n * PAGE, D_ROW)
+
+
 def mla_version() -> int:
     return lib().mla_version()
 

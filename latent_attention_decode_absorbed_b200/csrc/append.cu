@@ -1,4 +1,5 @@
-// Paged cache append: one warp writes one token's 576-number cache row.
+// Paged cache append: one warp writes one token's 576-number cache row (into
+// the page-blocked layout: nine contiguous [64 rows x 64 columns] blocks per page).
 //
 // "KV Compression - DeepSeek-V3", "How it works": the 576-wide wkv_a output is
 // split [512, 64]; the latent goes through RMSNorm and the rope part through
@@ -59,7 +60,7 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a) {
     for (int i = 0; i < 16; ++i) am = fmaxf(am, fabsf(c[i]));
     am = warp_max(am);
     const float q = am > 0.f ? 448.0f / am : 0.f;
-    uint8_t* dst = reinterpret_cast<uint8_t*>(a.cache) + slot * MLA_D_ROW;
+    uint8_t* dst = reinterpret_cast<uint8_t*>(a.cache);
     uint32_t w[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -67,29 +68,29 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a) {
       uint16_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c[4 * i + 2] * q, c[4 * i + 3] * q), __NV_SATFINITE, __NV_E4M3);
       w[i] = (uint32_t)lo | ((uint32_t)hi << 16);
     }
-    *reinterpret_cast<uint4*>(dst + 16 * lane) = make_uint4(w[0], w[1], w[2], w[3]);
+    *reinterpret_cast<uint4*>(dst + cache_index(slot, 16 * lane)) = make_uint4(w[0], w[1], w[2], w[3]);
     uint16_t rk = __nv_cvt_float2_to_fp8x2(make_float2(r0 * q, r1 * q), __NV_SATFINITE, __NV_E4M3);
-    *reinterpret_cast<uint16_t*>(dst + MLA_D_C + 2 * lane) = rk;
+    *reinterpret_cast<uint16_t*>(dst + cache_index(slot, MLA_D_C + 2 * lane)) = rk;
     if (lane == 0) a.cache_scale[slot] = am * (1.0f / 448.0f);
   } else if constexpr (CK == MLA_BF16) {
-    __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(a.cache) + slot * MLA_D_ROW;
+    __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(a.cache);
     uint32_t w[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       __nv_bfloat162 h = __floats2bfloat162_rn(c[2 * i], c[2 * i + 1]);
       w[i] = *reinterpret_cast<uint32_t*>(&h);
     }
-    uint4* d4 = reinterpret_cast<uint4*>(dst + 16 * lane);
+    uint4* d4 = reinterpret_cast<uint4*>(dst + cache_index(slot, 16 * lane));
     d4[0] = make_uint4(w[0], w[1], w[2], w[3]);
     d4[1] = make_uint4(w[4], w[5], w[6], w[7]);
     __nv_bfloat162 rk = __floats2bfloat162_rn(r0, r1);
-    *reinterpret_cast<__nv_bfloat162*>(dst + MLA_D_C + 2 * lane) = rk;
+    *reinterpret_cast<__nv_bfloat162*>(dst + cache_index(slot, MLA_D_C + 2 * lane)) = rk;
   } else {
-    float* dst = reinterpret_cast<float*>(a.cache) + slot * MLA_D_ROW;
-    float4* d4 = reinterpret_cast<float4*>(dst + 16 * lane);
+    float* dst = reinterpret_cast<float*>(a.cache);
+    float4* d4 = reinterpret_cast<float4*>(dst + cache_index(slot, 16 * lane));
 #pragma unroll
     for (int i = 0; i < 4; ++i) d4[i] = make_float4(c[4 * i], c[4 * i + 1], c[4 * i + 2], c[4 * i + 3]);
-    *reinterpret_cast<float2*>(dst + MLA_D_C + 2 * lane) = make_float2(r0, r1);
+    *reinterpret_cast<float2*>(dst + cache_index(slot, MLA_D_C + 2 * lane)) = make_float2(r0, r1);
   }
 }
 

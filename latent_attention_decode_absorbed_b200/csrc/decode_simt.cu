@@ -71,9 +71,10 @@ __global__ void __launch_bounds__(512) decode_simt_kernel(DecodeArgs a) {
       const long long sl = slot_of[jj];
       float v = 0.f;
       if (sl >= 0) {
-        if (CK == MLA_F32) v = reinterpret_cast<const float*>(a.cache)[sl * MLA_D_ROW + d];
-        else if (CK == MLA_BF16) v = to_f32(reinterpret_cast<const __nv_bfloat16*>(a.cache)[sl * MLA_D_ROW + d]);
-        else v = e4m3_to_f32(reinterpret_cast<const uint8_t*>(a.cache)[sl * MLA_D_ROW + d]) * scale_of[jj];
+        const size_t ci = cache_index((size_t)sl, d);
+        if (CK == MLA_F32) v = reinterpret_cast<const float*>(a.cache)[ci];
+        else if (CK == MLA_BF16) v = to_f32(reinterpret_cast<const __nv_bfloat16*>(a.cache)[ci]);
+        else v = e4m3_to_f32(reinterpret_cast<const uint8_t*>(a.cache)[ci]) * scale_of[jj];
       }
       tile[jj * MLA_D_ROW + d] = v;
     }

@@ -19,19 +19,24 @@
 // {[128r,128r+128), [256+128r, 256+128r+128)} of O^T in its TMEM.  TMEM per
 // CTA: two S^T buffers (2 x 128 columns) + O^T (2 x 128 columns) = 512.
 //
-// Cache rows stream through a ring of 16 KB shared-memory slots filled by TMA
-// (one 64-row page x 64 columns per 8 KB box, 128-byte swizzle).  The same
-// bytes serve as the K-major A operand of S^T (rows x dims) and the MN-major
-// A operand of O^T (dims x rows).  Warp roles per CTA: 0 TMA producer and
-// TMEM allocator, 1 MMA issuer (leader CTA only), 2-9 softmax (two
-// warpgroups, one per half of the heads; thread = cached row).
+// Cache rows stream through a ring of 16 KB shared-memory slots filled by
+// TMA (128-byte swizzle) in the order the MMA consumes them: S^T slots hold
+// [128 rows x 64 columns] K-major operands (one 8 KB box per page, issued by
+// two lanes), O^T slots hold [64 rows x this CTA's 128 dims] read as
+// MN-major operands (one 16 KB box); the O^T loads of the peer's rows hit
+// L2.  The pool is page-blocked, so every box is a contiguous read.
+// Warp roles per CTA: 0 TMA producer and TMEM allocator, 1 MMA issuer
+// (leader CTA only), 2-9 softmax (two warpgroups, one per half of the heads;
+// thread = cached row).
 //
 // Softmax per tile: each warp takes the per-head max of its 32 rows with
 // redux.sync, the 4 warps of a warpgroup combine through shared memory, the
 // pair exchanges its maxima through distributed shared memory, and the
 // running max only moves when the tile max exceeds it by more than 2^8 (the
 // accumulator is rescaled in TMEM then).  P = 2^(u - m) is written as bf16
-// straight into the P^T operand of the CTA that owns those heads.
+// straight into the P^T operand of the CTA that owns those heads.  The MMA
+// issuer keeps the score GEMM two tiles ahead of the value GEMM, so the
+// softmax of one tile overlaps the tensor work of the next ones.
 #include <math.h>
 
 #include "mla_device.cuh"
@@ -43,7 +48,7 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 320;             // 10 warps: see the role map above
 constexpr int kSlotBytes = 16384;
 constexpr int kBoxBytes = 8192;           // 64 rows x 128 bytes
 constexpr int kTile = 256;                // cached rows per pair tile
@@ -51,6 +56,7 @@ constexpr int kChunks = 9;                // 576 / 64 column chunks
 constexpr float kRescaleLog2 = 8.0f;      // lazy rescale threshold (log2 units)
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
+constexpr int kWarpProd = 0, kWarpMma = 1, kWarpSoft0 = 2;
 
 struct TcParams {
   int n_heads, q_len, batch;
@@ -67,17 +73,17 @@ struct TcParams {
 template <int NH>
 struct Layout {
   static constexpr int HPW = NH / 2;                      // heads per CTA / per warpgroup
-  static constexpr int kRingSlots = 7;
+  static constexpr int kSlots = 7;                        // ring of operand slots
   static constexpr int kQChunk = HPW * 128;               // one 64-column chunk of this CTA's Q rows
   static constexpr int kPChunk = HPW * 128;               // 64 rows of P^T for this CTA's heads
   static constexpr int kRing = 0;
-  static constexpr int kQ = kRing + kRingSlots * kSlotBytes;
+  static constexpr int kQ = kRing + kSlots * kSlotBytes;
   static constexpr int kP = kQ + kChunks * kQChunk;
   static constexpr int kMisc = kP + 4 * kPChunk;
   // misc area (bytes from kMisc)
   static constexpr int kBars = 0;                          // 64 barriers max
   static constexpr int kTmemSlot = 64 * 8;
-  static constexpr int kAbort = kTmemSlot + 4;      // +8, +12: per-warpgroup flags
+  static constexpr int kAbort = kTmemSlot + 4;             // +8, +12: per-warpgroup flags
   static constexpr int kMused = kTmemSlot + 32;            // float [2][NH]
   static constexpr int kRed = kMused + 2 * NH * 4;          // float [2 wg][4 warps][HPW]
   static constexpr int kOwnMax = kRed + 2 * 4 * HPW * 4;    // float [NH]
@@ -91,15 +97,16 @@ struct Layout {
 // barrier indices in the misc area
 template <int NS>
 struct Bars {
-  static constexpr int full = 0;               // [NS]  leader: TMA bytes of both CTAs
-  static constexpr int empty = NS;             // [NS]  both: MMA done with the slot
-  static constexpr int s_full = 2 * NS;        // [2]   both: S^T buffer ready
-  static constexpr int s_free = 2 * NS + 2;    // [2]   leader: both CTAs read the S^T buffer
-  static constexpr int p_full = 2 * NS + 4;    //       leader: both CTAs wrote P^T
-  static constexpr int o_done = 2 * NS + 5;    //       both: O^T MMAs of the tile done
-  static constexpr int mx_full = 2 * NS + 6;   // [2]   both: the peer's tile maxima arrived
-  static constexpr int q_full = 2 * NS + 8;    //       leader: Q of both CTAs loaded
-  static constexpr int l_full = 2 * NS + 9;    //       both: the peer's row sums arrived
+  static constexpr int full = 0;                     // [NS] leader: TMA bytes of both CTAs
+  static constexpr int empty = NS;                   // [NS] both: MMA done with the slot
+  static constexpr int base = 2 * NS;
+  static constexpr int s_full = base;                // [2]   both: S^T buffer ready
+  static constexpr int s_free = base + 2;            // [2]   leader: both CTAs loaded the S^T buffer
+  static constexpr int p_full = base + 4;            //       leader: both CTAs wrote P^T
+  static constexpr int o_done = base + 5;            //       both: O^T MMAs of the tile done
+  static constexpr int mx_full = base + 6;           // [2]   both: the peer's tile maxima arrived
+  static constexpr int q_full = base + 8;            //       leader: Q of both CTAs loaded
+  static constexpr int l_full = base + 9;            //       both: the peer's row sums arrived
 };
 
 __device__ __forceinline__ float redux_max(float v) {
@@ -149,19 +156,29 @@ __device__ __forceinline__ int page_of(const TcParams& p, int b, int row, bool* 
   return *ok ? pg : 0;
 }
 
+// The ring of operand slots shared by the pair: the leader's `full` barrier
+// counts the bytes both CTAs load; `empty` is arrived by the MMA commit in
+// both CTAs.  `kc` counts slots handed out, in the order the MMA uses them.
+struct Ring {
+  uint32_t base;      // shared address of slot 0
+  uint32_t full0;     // barrier of slot 0 (this CTA's address)
+  uint32_t empty0;
+  int slots;
+  uint32_t kc = 0;
+};
+
 template <int NH>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-    decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_constant__ CUtensorMap tm_q,
-                     const TcParams p) {
+    decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_constant__ CUtensorMap tm_cache2,
+                     const __grid_constant__ CUtensorMap tm_q, const TcParams p) {
   using LY = Layout<NH>;
   constexpr int HPW = LY::HPW;
-  constexpr int NS = LY::kRingSlots;
-  using B = Bars<NS>;
+  using B = Bars<LY::kSlots>;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t s_base = smem_u32(smem);
-  const uint32_t s_ring = s_base + LY::kRing, s_q = s_base + LY::kQ, s_p = s_base + LY::kP;
+  const uint32_t s_q = s_base + LY::kQ, s_p = s_base + LY::kP;
   uint8_t* misc = smem + LY::kMisc;
   const uint32_t s_misc = s_base + LY::kMisc;
   auto bar = [&](int i) -> uint32_t { return s_misc + LY::kBars + 8 * i; };
@@ -192,7 +209,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   // ---- set-up: barriers, TMEM, cluster sync
   if (threadIdx.x == 0) {
-    for (int i = 0; i < NS; ++i) {
+    for (int i = 0; i < LY::kSlots; ++i) {
       mbar_init(bar(B::full + i), 1);
       mbar_init(bar(B::empty + i), 1);
     }
@@ -209,12 +226,41 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     fence_mbar_init();
   }
   for (int i = threadIdx.x; i < 2 * NH; i += kThreads) m_used[i] = -INFINITY;
-  if (warp == 0) tmem_alloc_pair(s_misc + LY::kTmemSlot, kTmemCols);
+  if (warp == kWarpProd) tmem_alloc_pair(s_misc + LY::kTmemSlot, kTmemCols);
   tc_fence_before();
   cluster_sync();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(misc + LY::kTmemSlot);
 
+  Ring ring{s_base + LY::kRing, bar(B::full), bar(B::empty), LY::kSlots};
+
+  // producer side (whole warp): lane 0 waits for a free slot and posts the
+  // expected bytes (leader); the lanes then issue the slot's boxes
+  auto take = [&](Ring& rg, uint32_t& dst, uint32_t& fb) -> bool {
+    const uint32_t slot = rg.kc % rg.slots;
+    const uint32_t ph = (rg.kc / rg.slots) & 1u;
+    bool ok = true;
+    if (lane == 0) {
+      ok = mbar_wait(rg.empty0 + 8 * slot, ph ^ 1u, abort_flag);
+      if (ok && leader) mbar_arrive_expect_tx(rg.full0 + 8 * slot, 2u * kSlotBytes);
+    }
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    dst = rg.base + slot * kSlotBytes;
+    fb = mapa(rg.full0 + 8 * slot, 0);
+    ++rg.kc;
+    return ok;
+  };
+  // MMA side: wait for a filled slot
+  auto ready = [&](Ring& rg, uint32_t& src, uint32_t& empty) -> bool {
+    const uint32_t slot = rg.kc % rg.slots;
+    const uint32_t ph = (rg.kc / rg.slots) & 1u;
+    if (!mbar_wait(rg.full0 + 8 * slot, ph, abort_flag)) return false;
+    tc_fence_after();
+    src = rg.base + slot * kSlotBytes;
+    empty = rg.empty0 + 8 * slot;
+    ++rg.kc;
+    return true;
+  };
   if (n_tiles == 0) {
     // nothing visible in this split: o = 0, lse = -inf (heads split by rank)
     for (int i = threadIdx.x; i < p.n_heads * MLA_D_C; i += kThreads) {
@@ -223,74 +269,82 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       p.o_part[(((size_t)r * p.n_heads + h) * S + s) * MLA_D_C + d] = 0.f;
       if (d == 0) p.lse_part[((size_t)r * p.n_heads + h) * S + s] = -INFINITY;
     }
-  } else if (warp == 0) {
-    // ================= TMA producer (both CTAs) =================
+  } else if (warp == kWarpProd) {
+    // ============ TMA producer (both CTAs), in the order the MMA consumes ============
+    // S(0), S(1), then per tile i: S(i+2), O(i).  The pool is page-blocked
+    // (nine contiguous [64 rows x 64 columns] blocks per page), viewed as 2-D
+    // [blocks * 64 lines x 64 columns].  An S^T slot is block c of this CTA's
+    // two pages (two contiguous 8 KB boxes, lanes 0/1); an O^T slot is the two
+    // adjacent blocks of this CTA's 128 dims of one page (one contiguous 16 KB
+    // box).
     if (lane == 0) {
       tma_prefetch_desc(&tm_cache);
+      tma_prefetch_desc(&tm_cache2);
       tma_prefetch_desc(&tm_q);
       const uint32_t q_bar = mapa(bar(B::q_full), 0);
       if (leader) mbar_arrive_expect_tx(bar(B::q_full), 2u * kChunks * LY::kQChunk);
       for (int c = 0; c < kChunks; ++c)
         tma_load_3d_pair(s_q + c * LY::kQChunk, &tm_q, 64 * c, (int)rank * HPW, r, q_bar);
-      uint32_t kc = 0;
-      bool ok = true;
-      auto take_slot = [&](uint32_t& slot) -> bool {
-        slot = kc % NS;
-        const uint32_t ph = (kc / NS) & 1u;
-        if (!mbar_wait(bar(B::empty + slot), ph ^ 1u, abort_flag)) return false;
-        if (leader) mbar_arrive_expect_tx(bar(B::full + slot), 2u * kSlotBytes);
-        ++kc;
-        return true;
-      };
-      auto emit_o = [&](int j) -> bool {
-        for (int pg_i = 0; pg_i < 4; ++pg_i) {
-          const int row0 = lo + kTile * j + 64 * pg_i;
-          if (row0 >= hi) break;
-          bool vld;
-          const int pg = page_of(p, b, row0, &vld);
-          for (int bb = 0; bb < 2; ++bb) {
-            uint32_t slot;
-            if (!take_slot(slot)) return false;
-            const uint32_t dst = s_ring + slot * kSlotBytes;
-            const uint32_t fb = mapa(bar(B::full + slot), 0);
-            const int x0 = 256 * bb + 128 * (int)rank;
-            tma_load_2d_pair(dst, &tm_cache, x0, pg * 64, fb);
-            tma_load_2d_pair(dst + kBoxBytes, &tm_cache, x0 + 64, pg * 64, fb);
-          }
-        }
-        return true;
-      };
-      for (int i = 0; i < n_tiles && ok; ++i) {
-        const int row0 = lo + kTile * i + 128 * (int)rank;
-        bool v0, v1;
-        const int pg0 = page_of(p, b, row0, &v0);
-        const int pg1 = page_of(p, b, row0 + 64, &v1);
-        for (int c = 0; c < kChunks && ok; ++c) {
-          uint32_t slot;
-          if (!take_slot(slot)) { ok = false; break; }
-          const uint32_t dst = s_ring + slot * kSlotBytes;
-          const uint32_t fb = mapa(bar(B::full + slot), 0);
-          tma_load_2d_pair(dst, &tm_cache, 64 * c, pg0 * 64, fb);
-          tma_load_2d_pair(dst + kBoxBytes, &tm_cache, 64 * c, pg1 * 64, fb);
-        }
-        if (ok && i >= 1) ok = emit_o(i - 1);
-      }
-      if (ok) emit_o(n_tiles - 1);
     }
-  } else if (warp == 1) {
+    auto load_s = [&](int i) -> bool {
+      bool vv;
+      const int pg = page_of(p, b, lo + kTile * i + 128 * (int)rank + 64 * (lane & 1), &vv);
+      for (int c = 0; c < kChunks; ++c) {
+        uint32_t dst, fb;
+        if (!take(ring, dst, fb)) return false;
+        if (lane < 2) tma_load_2d_pair(dst + lane * kBoxBytes, &tm_cache, 0, (pg * kChunks + c) * 64, fb);
+      }
+      return true;
+    };
+    auto load_o = [&](int j) -> bool {
+      for (int pg_i = 0; pg_i < 4; ++pg_i) {
+        const int row0 = lo + kTile * j + 64 * pg_i;
+        if (row0 >= hi) break;
+        bool vld;
+        const int pg = page_of(p, b, row0, &vld);
+        for (int bb = 0; bb < 2; ++bb) {
+          uint32_t dst, fb;
+          if (!take(ring, dst, fb)) return false;
+          if (lane == 0)
+            tma_load_2d_pair(dst, &tm_cache2, 0, (pg * kChunks + (256 * bb + 128 * (int)rank) / 64) * 64, fb);
+        }
+      }
+      return true;
+    };
+    bool ok = load_s(0);
+    if (ok && n_tiles > 1) ok = load_s(1);
+    for (int i = 0; i < n_tiles && ok; ++i) {
+      if (i + 2 < n_tiles) ok = load_s(i + 2);
+      if (ok) ok = load_o(i);
+    }
+  } else if (warp == kWarpMma) {
     // ================= MMA issuer (leader CTA) =================
+    // order: S(0), S(1), then per tile i: S(i+2), O(i) -- the score GEMM runs
+    // two tiles ahead so the softmax of tile i overlaps S(i+1), O(i-1), S(i+2)
     if (leader && lane == 0) {
       constexpr uint32_t idS = idesc_f16(256, NH, false, false);
       constexpr uint32_t idO = idesc_f16(256, NH, true, false);
-      uint32_t kc = 0;
       bool ok = mbar_wait(bar(B::q_full), 0, abort_flag);
       tc_fence_after();
-      auto wait_slot = [&](uint32_t& slot) -> bool {
-        slot = kc % NS;
-        const uint32_t ph = (kc / NS) & 1u;
-        if (!mbar_wait(bar(B::full + slot), ph, abort_flag)) return false;
-        tc_fence_after();
-        ++kc;
+      auto issue_s = [&](int i) -> bool {
+        const int sb = i & 1;
+        if (i >= 2) {
+          if (!mbar_wait(bar(B::s_free + sb), ((i - 2) >> 1) & 1, abort_flag)) return false;
+          tc_fence_after();
+        }
+        const uint32_t d = tmem + (sb ? kColS1 : kColS0);
+        for (int c = 0; c < kChunks; ++c) {
+          uint32_t a0, empty;
+          if (!ready(ring, a0, empty)) return false;
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks) {
+            const uint64_t ad = smem_desc_sw128(a0 + ks * 32, 16, 1024);
+            const uint64_t bd = smem_desc_sw128(s_q + c * LY::kQChunk + ks * 32, 16, 1024);
+            mma_pair_f16(d, ad, bd, idS, (c | ks) != 0);
+          }
+          mma_commit_pair(empty, 0x3);
+        }
+        mma_commit_pair(bar(B::s_full + sb), 0x3);
         return true;
       };
       auto issue_o = [&](int j) -> bool {
@@ -299,53 +353,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int pg_i = 0; pg_i < 4; ++pg_i) {
           if (lo + kTile * j + 64 * pg_i >= hi) break;
           for (int bb = 0; bb < 2; ++bb) {
-            uint32_t slot;
-            if (!wait_slot(slot)) return false;
-            const uint32_t a0 = s_ring + slot * kSlotBytes;
+            uint32_t a0, empty;
+            if (!ready(ring, a0, empty)) return false;
+#pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
               const uint64_t ad = smem_desc_sw128(a0 + ks * 2048, kBoxBytes, 1024);
               const uint64_t bd = smem_desc_sw128(s_p + pg_i * LY::kPChunk + ks * 32, 16, 1024);
               mma_pair_f16(tmem + kColO + bb * 128, ad, bd, idO, (j | pg_i | ks) != 0);
             }
-            mma_commit_pair(bar(B::empty + slot), 0x3);
+            mma_commit_pair(empty, 0x3);
           }
         }
         mma_commit_pair(bar(B::o_done), 0x3);
         return true;
       };
+      if (ok) ok = issue_s(0);
+      if (ok && n_tiles > 1) ok = issue_s(1);
       for (int i = 0; i < n_tiles && ok; ++i) {
-        const int sb = i & 1;
-        if (i >= 2) {
-          if (!mbar_wait(bar(B::s_free + sb), ((i - 2) >> 1) & 1, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-        }
-        const uint32_t d = tmem + (sb ? kColS1 : kColS0);
-        for (int c = 0; c < kChunks; ++c) {
-          uint32_t slot;
-          if (!wait_slot(slot)) { ok = false; break; }
-          const uint32_t a0 = s_ring + slot * kSlotBytes;
-          for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t ad = smem_desc_sw128(a0 + ks * 32, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(s_q + c * LY::kQChunk + ks * 32, 16, 1024);
-            mma_pair_f16(d, ad, bd, idS, (c | ks) != 0);
-          }
-          mma_commit_pair(bar(B::empty + slot), 0x3);
-        }
-        if (!ok) break;
-        mma_commit_pair(bar(B::s_full + sb), 0x3);
-        if (i >= 1) ok = issue_o(i - 1);
+        if (i + 2 < n_tiles) ok = issue_s(i + 2);
+        if (ok) ok = issue_o(i);
       }
-      if (ok) issue_o(n_tiles - 1);
     }
-  } else if (warp >= 2) {
-    // ================= softmax (both CTAs, 8 warps) =================
-    // Per tile, in column chunks of C heads so that few registers are live:
-    //   A  tile max per head (redux over a warp's rows, then over 4 warps)
+  } else {
+    // ================= softmax (both CTAs, warps 2-9) =================
+    // Per tile:
+    //   A  load the tile's scores (thread = row, HPW heads) into registers and
+    //      release the S^T buffer; per-head max over the warp (redux), then
+    //      over the 4 warps of the group
     //   -- warp 0 of the group exchanges maxima with the peer and sets the
     //      new running max (and the rescale factors) in shared memory
     //   B  P = 2^(u - m) written to P^T, running row sums updated
     constexpr int C = HPW < 32 ? HPW : 32;
-    const int g = (warp - 2) >> 2;             // warpgroup: heads [g*HPW, (g+1)*HPW)
+    const int g = (warp - kWarpSoft0) >> 2;    // warpgroup: heads [g*HPW, (g+1)*HPW)
     const int q = warp & 3;                    // TMEM lane quadrant
     const int tok = 32 * q + lane;             // row within this CTA's half of the tile
     const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
@@ -358,14 +397,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     float l_acc[HPW / C];
 #pragma unroll
     for (int k = 0; k < HPW / C; ++k) l_acc[k] = 0.f;
+    const int kt = 128 * (int)rank + tok;      // row within the pair tile
+    const int ke = kt & ~1;
+    const int wcol = ke & 63;
+    const uint32_t row_base = (ke >> 6) * LY::kPChunk + (wcol & 7) * 2;
     bool ok = true;
     for (int i = 0; i < n_tiles; ++i) {
       const int sb = i & 1;
       ok = __all_sync(0xffffffffu, mbar_wait(bar(B::s_full + sb), (i >> 1) & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      const uint32_t sc = tmem + lane_addr + (sb ? kColS1 : kColS0) + g * HPW;
-      const int row = lo + kTile * i + 128 * (int)rank + tok;
+      const int row = lo + kTile * i + kt;
       bool vld = row < hi;
       if (vld) {
         bool pok;
@@ -373,17 +415,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (!pok) { vld = false; flag_error(p.err, MLA_DEVERR_PAGE); }
       }
       const float sl = vld ? p.scale_log2 : 0.f;
-      // ---- A: per-head tile max
+      // ---- A: scores into registers, release the buffer, per-head tile max
+      float u[HPW];
+      {
+        const uint32_t sc = tmem + lane_addr + (sb ? kColS1 : kColS0) + g * HPW;
 #pragma unroll
-      for (int k = 0; k < HPW / C; ++k) {
-        float u[C];
-        tmem_ld<C>(sc + C * k, u);
+        for (int k = 0; k < HPW / C; ++k) tmem_ld<C>(sc + C * k, u + C * k);
         tmem_wait_ld();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa(bar(B::s_free + sb), 0));
 #pragma unroll
-        for (int h = 0; h < C; ++h) {
-          const float mx = redux_max(vld ? u[h] * sl : -INFINITY);
-          if (lane == (h & 31)) red_g[q * HPW + C * k + h] = mx;
-        }
+      for (int h = 0; h < HPW; ++h) {
+        u[h] = vld ? u[h] * sl : -INFINITY;
+        const float mx = redux_max(u[h]);
+        if (lane == (h & 31)) red_g[q * HPW + h] = mx;
       }
       named_barrier(1 + g, 128);
       const int xb = i & 1;
@@ -405,7 +452,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const float mn = (mt > mo + kRescaleLog2) ? mt : mo;
             m_next[h] = mn;
             // rescale factor for sums and accumulator kept so far (0 when nothing was kept)
-            alpha[g * HPW + h] = (mo == -INFINITY) ? 0.f : exp2f(mo - mn);
+            alpha[g * HPW + h] = (mo == -INFINITY) ? 0.f : exp2_approx(mo - mn);
             ch |= (mn != mo);
           }
           ch = __any_sync(0xffffffffu, ch);
@@ -415,64 +462,57 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       named_barrier(1 + g, 128);
       if (*abort_flag) { ok = false; break; }
       const bool changed = *changed_flag != 0;
+      // ---- B1: probabilities (fp32, in registers)
+#pragma unroll
+      for (int h = 0; h < HPW; ++h) {
+        const float mn = m_next[h];
+        u[h] = exp2_approx(u[h] - (mn == -INFINITY ? 0.f : mn));
+      }
       // the previous tile's O^T MMAs must be done: P^T buffer reuse and rescale
       if (i >= 1) {
         ok = __all_sync(0xffffffffu, mbar_wait(bar(B::o_done), (i - 1) & 1, abort_flag));
         if (!ok) break;
         tc_fence_after();
         if (changed) {
-#pragma unroll
+          constexpr int CC = C < 16 ? C : 16;
+#pragma unroll 1
           for (int bb = 0; bb < 2; ++bb) {
-#pragma unroll
-            for (int k = 0; k < HPW / C; ++k) {
-              const uint32_t oc = tmem + lane_addr + kColO + bb * 128 + g * HPW + C * k;
-              float o[C];
-              tmem_ld<C>(oc, o);
+#pragma unroll 1
+            for (int k = 0; k < HPW / CC; ++k) {
+              const uint32_t oc = tmem + lane_addr + kColO + bb * 128 + g * HPW + CC * k;
+              float o[CC];
+              tmem_ld<CC>(oc, o);
               tmem_wait_ld();
 #pragma unroll
-              for (int h = 0; h < C; ++h) o[h] *= alpha[g * HPW + C * k + h];
-              tmem_st<C>(oc, o);
+              for (int h = 0; h < CC; ++h) o[h] *= alpha[g * HPW + CC * k + h];
+              tmem_st<CC>(oc, o);
             }
           }
           tmem_wait_st();
         }
       }
-      // ---- B: probabilities, row sums, P^T (bf16, pairs of rows per 32-bit store)
-      const int kt = 128 * (int)rank + tok;
-      const int ke = kt & ~1;
-      const int w = ke & 63;
-      const uint32_t row_base = (ke >> 6) * LY::kPChunk + (w & 7) * 2;
+      // ---- B2: P^T (bf16, pairs of rows per 32-bit store), running row sums
 #pragma unroll
       for (int k = 0; k < HPW / C; ++k) {
-        float u[C];
-        tmem_ld<C>(sc + C * k, u);
-        tmem_wait_ld();
-#pragma unroll
-        for (int h = 0; h < C; ++h) {
-          const float mn = m_next[C * k + h];
-          u[h] = vld ? exp2f(u[h] * sl - (mn == -INFINITY ? 0.f : mn)) : 0.f;
-        }
+        float* uk = u + C * k;
 #pragma unroll
         for (int h = 0; h < C; h += 2) {
-          const float send = (lane & 1) ? u[h] : u[h + 1];
+          const float send = (lane & 1) ? uk[h] : uk[h + 1];
           const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
           const int hr = C * k + ((lane & 1) ? h + 1 : h);
-          __nv_bfloat162 pk = (lane & 1) ? __floats2bfloat162_rn(recv, u[h + 1]) : __floats2bfloat162_rn(u[h], recv);
+          __nv_bfloat162 pk = (lane & 1) ? __floats2bfloat162_rn(recv, uk[h + 1]) : __floats2bfloat162_rn(uk[h], recv);
           const uint32_t val = *reinterpret_cast<uint32_t*>(&pk);
-          const uint32_t off = row_base + hr * 128 + ((((w >> 3) ^ (hr & 7))) << 4);
+          const uint32_t off = row_base + hr * 128 + ((((wcol >> 3) ^ (hr & 7))) << 4);
           if (p_remote) st_cluster_b32(p_dst + off, val);
           else asm volatile("st.shared.b32 [%0], %1;" ::"r"(p_dst + off), "r"(val) : "memory");
         }
-        const float ls = transpose_reduce<C>(u, lane);
+        const float ls = transpose_reduce<C>(uk, lane);
         l_acc[k] = changed ? fmaf(l_acc[k], alpha[g * HPW + C * k + (lane % C)], ls) : l_acc[k] + ls;
       }
       tc_fence_before();
       fence_proxy_async_cluster();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive_cluster(mapa(bar(B::s_free + sb), 0));
-        mbar_arrive_cluster(mapa(bar(B::p_full), 0));
-      }
+      if (lane == 0) mbar_arrive_cluster(mapa(bar(B::p_full), 0));
     }
     // ---- epilogue: normalise O^T by the row sums, write o_part and lse
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(B::o_done), (n_tiles - 1) & 1, abort_flag));
@@ -538,7 +578,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   cluster_sync();
-  if (warp == 0) {
+  if (warp == kWarpProd) {
     tc_fence_after();
     tmem_dealloc_pair(tmem, kTmemCols);
   }
@@ -564,7 +604,8 @@ EncodeTiledFn encode_fn() {
 }
 
 template <int NH>
-cudaError_t launch_nh(const DecodeArgs& a, const CUtensorMap& tc, const CUtensorMap& tq, cudaStream_t st) {
+cudaError_t launch_nh(const DecodeArgs& a, const CUtensorMap& tc, const CUtensorMap& tc2, const CUtensorMap& tq,
+                      cudaStream_t st) {
   using LY = Layout<NH>;
   cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<NH>, cudaFuncAttributeMaxDynamicSharedMemorySize, LY::kSmem);
   if (e != cudaSuccess) return e;
@@ -572,7 +613,7 @@ cudaError_t launch_nh(const DecodeArgs& a, const CUtensorMap& tc, const CUtensor
              a.split_tokens, a.softmax_scale * 1.4426950408889634f, a.o_part, a.lse_part, a.err};
   const long long units = (long long)a.batch * a.q_len * a.num_splits;
   dim3 grid((unsigned)(2 * units));
-  decode_tc_kernel<NH><<<grid, kThreads, LY::kSmem, st>>>(tc, tq, p);
+  decode_tc_kernel<NH><<<grid, kThreads, LY::kSmem, st>>>(tc, tc2, tq, p);
   return cudaGetLastError();
 }
 
@@ -588,14 +629,16 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st) {
   if (!enc) return cudaErrorNotSupported;
   const int NH = a.n_heads <= 16 ? 16 : a.n_heads <= 32 ? 32 : a.n_heads <= 64 ? 64 : 128;
   const int HPW = NH / 2;
-  CUtensorMap tc, tq;
-  {
-    cuuint64_t dims[2] = {MLA_D_ROW, (cuuint64_t)a.num_pages * 64};
-    cuuint64_t strides[1] = {MLA_D_ROW * 2};
-    cuuint32_t box[2] = {64, 64};
+  CUtensorMap tc, tc2, tq;
+  // the page-blocked pool as 2-D [num_pages * 9 * 64 lines x 64 columns], 128-byte lines:
+  // boxes of 64 lines (one block) and of 128 lines (two adjacent blocks)
+  for (int k = 0; k < 2; ++k) {
+    cuuint64_t dims[2] = {64, (cuuint64_t)a.num_pages * kChunks * 64};
+    cuuint64_t strides[1] = {128};
+    cuuint32_t box[2] = {64, k == 0 ? 64u : 128u};
     cuuint32_t es[2] = {1, 1};
-    if (enc(&tc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a.cache), dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+    if (enc(k == 0 ? &tc : &tc2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a.cache), dims, strides, box,
+            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
@@ -610,10 +653,10 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st) {
       return cudaErrorInvalidValue;
   }
   switch (NH) {
-    case 16: return launch_nh<16>(a, tc, tq, st);
-    case 32: return launch_nh<32>(a, tc, tq, st);
-    case 64: return launch_nh<64>(a, tc, tq, st);
-    default: return launch_nh<128>(a, tc, tq, st);
+    case 16: return launch_nh<16>(a, tc, tc2, tq, st);
+    case 32: return launch_nh<32>(a, tc, tc2, tq, st);
+    case 64: return launch_nh<64>(a, tc, tc2, tq, st);
+    default: return launch_nh<128>(a, tc, tc2, tq, st);
   }
 }
 

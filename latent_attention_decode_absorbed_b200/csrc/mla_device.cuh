@@ -23,6 +23,15 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 
+// Page-blocked cache layout: a 64-row page is stored as nine blocks of
+// [64 rows x 64 columns], block c holding columns 64c..64c+63, so every
+// block is contiguous in memory.  Element index of (slot = page*64 + row, d).
+__device__ __forceinline__ size_t cache_index(size_t slot, int d) {
+  const size_t page = slot >> 6;
+  const int row = static_cast<int>(slot & 63);
+  return ((page * (MLA_D_ROW / 64) + (d >> 6)) * 64 + row) * 64 + (d & 63);
+}
+
 __device__ __forceinline__ void flag_error(int32_t* err, int32_t bits) {
   if (err) atomicOr(err, bits);
 }

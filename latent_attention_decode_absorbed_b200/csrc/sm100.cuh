@@ -64,31 +64,47 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
   asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
                : "memory");
 }
+// Test for completion of the phase with the given parity.  Cluster scope
+// (needed when the arrivals carry another CTA's writes) costs several times
+// the CTA-scope form, so each wait names the scope it needs.
+template <bool kCluster = true>
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
+  if constexpr (kCluster)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+  else
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
   return ok != 0;
 }
 
 // Wait until the phase with the given parity has completed.  Gives up after
-// `limit_ns` (or as soon as *abort is set by another thread), sets *abort and
-// returns false.  Every wait in the tensor-core kernels goes through here.
+// `limit_cycles` SM clock cycles (about 2 s at 2 GHz), or as soon as *abort is
+// set by another thread, sets *abort and returns false.  Every wait in the
+// tensor-core kernels goes through here.  The bound uses the SM cycle counter:
+// it is cheap to read on every slow-path iteration, unlike the global timer.
+template <bool kCluster = true>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
-                                          uint64_t limit_ns = 1000000000ull) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer();
+                                          uint64_t limit_cycles = 4000000000ull) {
+  if (mbar_try_wait<kCluster>(bar, parity)) return true;
+  const uint64_t t0 = clock64();
   uint32_t n = 0;
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((++n & 63u) == 0) {
+    if (mbar_try_wait<kCluster>(bar, parity)) return true;
+    if ((++n & 255u) == 0) {
       if (*abort) return false;
-      if (globaltimer() - t0 > limit_ns) {
+      if (clock64() - t0 > limit_cycles) {
         *abort = 1;
         return false;
       }
@@ -104,6 +120,12 @@ __device__ __forceinline__ void fence_proxy_async_cluster() {
 }
 
 // ---------------------------------------------------------------- TMA
+// Bring `bytes` (a multiple of 16) of global memory into L2, asynchronously.
+__device__ __forceinline__ void prefetch_l2(const void* gaddr, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(gaddr)), "r"(bytes)
+               : "memory");
+}
+
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -164,6 +186,13 @@ __device__ __forceinline__ void mma_commit_pair(uint32_t bar, uint16_t mask) {
       "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
       "h"(mask)
       : "memory");
+}
+
+// 2^x on the MUFU unit (ex2.approx, flush-to-zero; relative error ~2^-22).
+__device__ __forceinline__ float exp2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }

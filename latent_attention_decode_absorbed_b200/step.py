@@ -56,7 +56,8 @@ class DecodeStep:
             np.asarray(norm_gain, np.float32)).to(self.device)
         dev = self.device
         # zero-filled: the tensor-core decode reads whole pages (see mla_decode_fwd)
-        self.cache = torch.zeros((self.num_pages, PAGE, D_ROW), dtype=_torch_dtype(self.cache_dtype), device=dev)
+        self.cache = torch.zeros((self.num_pages, D_ROW // 64, PAGE, 64), dtype=_torch_dtype(self.cache_dtype),
+                                 device=dev)
         self.cache_scale = (torch.zeros((self.num_pages, PAGE), dtype=torch.float32, device=dev)
                             if self.cache_dtype == MLA_E4M3 else None)
         rows = self.batch * self.q_len

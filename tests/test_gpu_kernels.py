@@ -59,7 +59,7 @@ def test_append_exact(cache_dt, kv_dt):
     eps = 1e-6
     max_pos = 200
     cos, sin = _rope_tables(max_pos)
-    cache = torch.full((num_pages, 64, 576), 0xFF if cache_dt == "e4m3" else 0, dtype=TDT[cache_dt], device="cuda")
+    cache = torch.zeros((num_pages, 9, 64, 64), dtype=TDT[cache_dt], device="cuda")
     cache.view(torch.uint8).fill_(0xFF)                     # sentinel: every byte 0xFF
     scale = torch.full((num_pages, 64), float("nan"), device="cuda") if cache_dt == "e4m3" else None
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
@@ -69,7 +69,8 @@ def test_append_exact(cache_dt, kv_dt):
                          num_pages, err)
     torch.cuda.synchronize()
     assert int(err.item()) == 0
-    raw = cache.view(torch.uint8).cpu().numpy().reshape(num_pages * 64, -1)
+    rows_dev = mla.unpack_cache_rows(cache)                  # logical rows [num_pages*64, 576]
+    raw = rows_dev.contiguous().view(torch.uint8).cpu().numpy().reshape(num_pages * 64, -1)
     slot = bt[seq, pos // 64].astype(np.int64) * 64 + pos % 64
     # indexing: exactly the appended slots changed
     touched = np.zeros(num_pages * 64, bool); touched[slot] = True
@@ -77,14 +78,14 @@ def test_append_exact(cache_dt, kv_dt):
     assert not np.any(np.all(raw[touched] == 0xFF, axis=1))
     ref = oracle.cache_rows(kv, pos, gain, eps)              # fp64 [n, 576]
     if cache_dt == "f32":
-        got = cache.view(-1, 576).cpu().numpy().astype(np.float64)[slot]
+        got = rows_dev.cpu().numpy().astype(np.float64)[slot]
         np.testing.assert_allclose(got, ref, rtol=2e-6, atol=1e-6)
     elif cache_dt == "bf16":
-        got = cache.view(-1, 576).to(torch.float64).cpu().numpy()[slot]
+        got = rows_dev.to(torch.float64).cpu().numpy()[slot]
         bad = bf16_exact_or_boundary(got, ref)
         assert not bad.any(), f"{bad.sum()} bf16 values off (first at {np.argwhere(bad)[:3]})"
     else:
-        codes = cache.view(-1, 576).cpu().numpy()[slot]
+        codes = rows_dev.cpu().numpy()[slot]
         sc = scale.view(-1).cpu().numpy().astype(np.float64)
         assert np.all(np.isnan(np.delete(sc, slot)))
         ref_codes, ref_scale = oracle.quantize_rows_e4m3(ref)
@@ -104,7 +105,7 @@ def test_append_bad_indices_are_skipped_and_flagged():
     bt, num_pages = _pool(lens, spare=0, seed=3)
     bt[1, 0] = num_pages + 5                                # a page outside the pool
     cos, sin = _rope_tables(128)
-    cache = torch.zeros((num_pages, 64, 576), dtype=torch.bfloat16, device="cuda")
+    cache = torch.zeros((num_pages, 9, 64, 64), dtype=torch.bfloat16, device="cuda")
     cache.view(torch.uint8).fill_(0xFF)
     kv = to_device(round_bf16(np.ones((4, 576), np.float32)), "bf16")
     for seq, pos, flag in [([0, 0, 0, 0], [0, 1, 64, 2], mla.MLA_DEVERR_POSITION),   # 64 is past the table
@@ -118,7 +119,7 @@ def test_append_bad_indices_are_skipped_and_flagged():
                              num_pages, err)
         torch.cuda.synchronize()
         assert int(err.item()) & flag
-        raw = cache.view(torch.uint8).view(num_pages * 64, -1).cpu().numpy()
+        raw = mla.unpack_cache_rows(cache).contiguous().view(torch.uint8).cpu().numpy()
         good = [(s, p) for s, p in zip(seq, pos) if s < 2 and p < 64 and not (s == 1)]
         n_written = int(np.sum(~np.all(raw == 0xFF, axis=1)))
         assert n_written == len(good)
@@ -186,13 +187,13 @@ def _random_cache(g, num_pages, cache_dt):
     x = g.standard_normal((num_pages * 64, 576)).astype(np.float32)
     if cache_dt == "bf16":
         v = round_bf16(x)
-        return to_device(v, "bf16").view(num_pages, 64, 576), None, v.astype(np.float64)
+        return mla.pack_cache_rows(to_device(v, "bf16")), None, v.astype(np.float64)
     if cache_dt == "f32":
-        return to_device(x, "f32").view(num_pages, 64, 576), None, x.astype(np.float64)
+        return mla.pack_cache_rows(to_device(x, "f32")), None, x.astype(np.float64)
     codes = torch.from_numpy(np.clip(x * 100, -440, 440)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
     sc = (g.uniform(0.002, 0.02, num_pages * 64)).astype(np.float32)
     vals = oracle.e4m3_decode(codes) * sc.astype(np.float64)[:, None]
-    return (torch.from_numpy(codes).cuda().view(num_pages, 64, 576), torch.from_numpy(sc).cuda(), vals)
+    return (mla.pack_cache_rows(torch.from_numpy(codes).cuda()), torch.from_numpy(sc).cuda(), vals)
 
 
 CASES = [

@@ -33,7 +33,7 @@ def _problem(seed, lens, T, H, split_tokens):
     cache = to_device(round_bf16(g.standard_normal((num_pages * 64, 576)).astype(np.float32)), "bf16")
     q = to_device(round_bf16(g.standard_normal((len(lens) * T, H, 576)).astype(np.float32) * 0.25), "bf16")
     S = -(-bt.shape[1] * 64 // split_tokens)
-    return dict(q_abs=q, q_dtype=mla.MLA_BF16, cache=cache.view(num_pages, 64, 576), cache_scale=None,
+    return dict(q_abs=q, q_dtype=mla.MLA_BF16, cache=mla.pack_cache_rows(cache), cache_scale=None,
                 cache_dtype=mla.MLA_BF16, num_pages=num_pages, block_table=torch.from_numpy(bt).cuda(),
                 max_pages_per_seq=bt.shape[1], page_size=64,
                 seq_lens=torch.tensor(lens, dtype=torch.int32).cuda(), batch=len(lens), q_len=T, n_heads=H,
