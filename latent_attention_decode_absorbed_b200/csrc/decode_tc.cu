@@ -19,11 +19,14 @@
 // {[128r,128r+128), [256+128r, 256+128r+128)} of O^T in its TMEM.  TMEM per
 // CTA: two S^T buffers (2 x 128 columns) + O^T (2 x 128 columns) = 512.
 //
-// Cache rows stream through a ring of 16 KB shared-memory slots filled by
-// TMA (128-byte swizzle) in the order the MMA consumes them: S^T slots hold
-// [128 rows x 64 columns] K-major operands (one 8 KB box per page, issued by
-// two lanes), O^T slots hold [64 rows x this CTA's 128 dims] read as
-// MN-major operands (one 16 KB box); the O^T loads of the peer's rows hit
+// Cache rows stream through a ring of 32 KB shared-memory stages filled by
+// TMA (128-byte swizzle) in the order the MMA consumes them.  A stage costs a
+// fixed handshake (barrier wait, expected-bytes post, commit) whatever its
+// size, and 16 KB stages cannot keep up with HBM, so a stage carries two
+// column chunks of the score operand (four 8 KB boxes: [128 rows x 64
+// columns] K-major per chunk, one box per page, issued by four lanes) or one
+// page of the value operand (two 16 KB boxes: [64 rows x this CTA's 128 dims]
+// read MN-major, one per dims block); the value loads of the peer's rows hit
 // L2.  The pool is page-blocked, so every box is a contiguous read.
 // Warp roles per CTA: 0 TMA producer and TMEM allocator, 1 MMA issuer
 // (leader CTA only), 2-9 softmax (two warpgroups, one per half of the heads;
@@ -48,9 +51,13 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 320;             // 10 warps: see the role map above
-constexpr int kSlotBytes = 16384;
+constexpr int kSoftGroups = 4;           // softmax warpgroups, each a quarter of the heads
+constexpr int kThreads = 32 * (2 + 4 * kSoftGroups);  // 18 warps: see the role map above
+constexpr int kSlotBytes = 32768;         // one ring stage
 constexpr int kBoxBytes = 8192;           // 64 rows x 128 bytes
+constexpr int kChunkBytes = 16384;        // one column chunk of 128 rows (both pages)
+constexpr int kSStages = 5;               // score stages per tile: chunks {0,1} {2,3} {4,5} {6,7} {8}
+
 constexpr int kTile = 256;                // cached rows per pair tile
 constexpr int kChunks = 9;                // 576 / 64 column chunks
 constexpr float kRescaleLog2 = 8.0f;      // lazy rescale threshold (log2 units)
@@ -72,26 +79,33 @@ struct TcParams {
 
 template <int NH>
 struct Layout {
-  static constexpr int HPW = NH / 2;                      // heads per CTA / per warpgroup
-  static constexpr int kSlots = 7;                        // ring of operand slots
+  static constexpr int HPW = NH / 2;                      // heads per CTA (its half of Q and P^T)
+  static constexpr int HPG = NH / kSoftGroups;            // heads per softmax warpgroup
   static constexpr int kQChunk = HPW * 128;               // one 64-column chunk of this CTA's Q rows
   static constexpr int kPChunk = HPW * 128;               // 64 rows of P^T for this CTA's heads
-  static constexpr int kRing = 0;
-  static constexpr int kQ = kRing + kSlots * kSlotBytes;
-  static constexpr int kP = kQ + kChunks * kQChunk;
-  static constexpr int kMisc = kP + 4 * kPChunk;
+  static constexpr int kPSlots = 6;                       // ring of P^T chunks (1.5 tiles)
   // misc area (bytes from kMisc)
   static constexpr int kBars = 0;                          // 64 barriers max
   static constexpr int kTmemSlot = 64 * 8;
-  static constexpr int kAbort = kTmemSlot + 4;             // +8, +12: per-warpgroup flags
+  static constexpr int kAbort = kTmemSlot + 4;
+  static constexpr int kChanged = kTmemSlot + 16;          // int [kSoftGroups]: running max moved
   static constexpr int kMused = kTmemSlot + 32;            // float [2][NH]
-  static constexpr int kRed = kMused + 2 * NH * 4;          // float [2 wg][4 warps][HPW]
-  static constexpr int kOwnMax = kRed + 2 * 4 * HPW * 4;    // float [NH]
+  static constexpr int kRed = kMused + 2 * NH * 4;          // float [kSoftGroups][4 warps][HPG]
+  static constexpr int kOwnMax = kRed + kSoftGroups * 4 * HPG * 4;  // float [NH]
   static constexpr int kXMax = kOwnMax + NH * 4;            // float [2][NH]   written by the peer
   static constexpr int kLOwn = kXMax + 2 * NH * 4;          // float [NH]
   static constexpr int kLX = kLOwn + NH * 4;                // float [NH]      written by the peer
   static constexpr int kMiscBytes = kLX + NH * 4;
+  // ring of operand stages: as many as fit next to Q, P^T and the misc area (at most 6)
+  static constexpr int kFixed = kChunks * kQChunk + kPSlots * kPChunk + kMiscBytes + 1024;
+  static constexpr int kFit = (227 * 1024 - kFixed) / kSlotBytes;
+  static constexpr int kSlots = kFit > 6 ? 6 : kFit;
+  static constexpr int kRing = 0;
+  static constexpr int kQ = kRing + kSlots * kSlotBytes;
+  static constexpr int kP = kQ + kChunks * kQChunk;
+  static constexpr int kMisc = kP + kPSlots * kPChunk;
   static constexpr int kSmem = kMisc + kMiscBytes + 1024;  // + alignment slack
+  static_assert(kSmem <= 227 * 1024 && kSlots >= 2, "shared memory budget");
 };
 
 // barrier indices in the misc area
@@ -107,6 +121,7 @@ struct Bars {
   static constexpr int mx_full = base + 6;           // [2]   both: the peer's tile maxima arrived
   static constexpr int q_full = base + 8;            //       leader: Q of both CTAs loaded
   static constexpr int l_full = base + 9;            //       both: the peer's row sums arrived
+  static constexpr int p_free = base + 10;           // [6]   both: O^T MMAs done with a P^T chunk slot
 };
 
 __device__ __forceinline__ float redux_max(float v) {
@@ -174,6 +189,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   using LY = Layout<NH>;
   constexpr int HPW = LY::HPW;
   using B = Bars<LY::kSlots>;
+  static_assert(B::base + 16 <= 64, "barrier area");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -215,13 +231,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(B::s_full + i), 1);
-      mbar_init(bar(B::s_free + i), 16);
-      mbar_init(bar(B::mx_full + i), 2);
+      mbar_init(bar(B::s_free + i), 2 * 4 * kSoftGroups);
+      mbar_init(bar(B::mx_full + i), kSoftGroups);
     }
-    mbar_init(bar(B::p_full), 16);
+    mbar_init(bar(B::p_full), 2 * 4 * kSoftGroups);
     mbar_init(bar(B::o_done), 1);
     mbar_init(bar(B::q_full), 1);
-    mbar_init(bar(B::l_full), 2);
+    mbar_init(bar(B::l_full), kSoftGroups);
+    for (int i = 0; i < LY::kPSlots; ++i) mbar_init(bar(B::p_free + i), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -236,13 +253,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   // producer side (whole warp): lane 0 waits for a free slot and posts the
   // expected bytes (leader); the lanes then issue the slot's boxes
-  auto take = [&](Ring& rg, uint32_t& dst, uint32_t& fb) -> bool {
+  auto take = [&](Ring& rg, uint32_t bytes, uint32_t& dst, uint32_t& fb) -> bool {
     const uint32_t slot = rg.kc % rg.slots;
     const uint32_t ph = (rg.kc / rg.slots) & 1u;
     bool ok = true;
     if (lane == 0) {
-      ok = mbar_wait(rg.empty0 + 8 * slot, ph ^ 1u, abort_flag);
-      if (ok && leader) mbar_arrive_expect_tx(rg.full0 + 8 * slot, 2u * kSlotBytes);
+      ok = mbar_wait<false>(rg.empty0 + 8 * slot, ph ^ 1u, abort_flag);
+      if (ok && leader) mbar_arrive_expect_tx(rg.full0 + 8 * slot, 2u * bytes);
     }
     ok = __shfl_sync(0xffffffffu, ok, 0);
     dst = rg.base + slot * kSlotBytes;
@@ -254,7 +271,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   auto ready = [&](Ring& rg, uint32_t& src, uint32_t& empty) -> bool {
     const uint32_t slot = rg.kc % rg.slots;
     const uint32_t ph = (rg.kc / rg.slots) & 1u;
-    if (!mbar_wait(rg.full0 + 8 * slot, ph, abort_flag)) return false;
+    if (!mbar_wait<false>(rg.full0 + 8 * slot, ph, abort_flag)) return false;
     tc_fence_after();
     src = rg.base + slot * kSlotBytes;
     empty = rg.empty0 + 8 * slot;
@@ -273,10 +290,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // ============ TMA producer (both CTAs), in the order the MMA consumes ============
     // S(0), S(1), then per tile i: S(i+2), O(i).  The pool is page-blocked
     // (nine contiguous [64 rows x 64 columns] blocks per page), viewed as 2-D
-    // [blocks * 64 lines x 64 columns].  An S^T slot is block c of this CTA's
-    // two pages (two contiguous 8 KB boxes, lanes 0/1); an O^T slot is the two
-    // adjacent blocks of this CTA's 128 dims of one page (one contiguous 16 KB
-    // box).
+    // [blocks * 64 lines x 64 columns].  A score stage is blocks c, c+1 of this
+    // CTA's two pages (lane l: block c + l/2 of page l%2, 8 KB each); a value
+    // stage is one page's two dims blocks of this CTA (lane l: dims block l,
+    // one contiguous 16 KB box each).  One ring in consumption order keeps the
+    // most bytes in flight: separate score and value rings measured slower.
     if (lane == 0) {
       tma_prefetch_desc(&tm_cache);
       tma_prefetch_desc(&tm_cache2);
@@ -289,10 +307,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     auto load_s = [&](int i) -> bool {
       bool vv;
       const int pg = page_of(p, b, lo + kTile * i + 128 * (int)rank + 64 * (lane & 1), &vv);
-      for (int c = 0; c < kChunks; ++c) {
+      for (int st = 0; st < kSStages; ++st) {
+        const int nc = st < kSStages - 1 ? 2 : 1;
         uint32_t dst, fb;
-        if (!take(ring, dst, fb)) return false;
-        if (lane < 2) tma_load_2d_pair(dst + lane * kBoxBytes, &tm_cache, 0, (pg * kChunks + c) * 64, fb);
+        if (!take(ring, nc * kChunkBytes, dst, fb)) return false;
+        if (lane < 2 * nc)
+          tma_load_2d_pair(dst + (lane >> 1) * kChunkBytes + (lane & 1) * kBoxBytes, &tm_cache, 0,
+                           (pg * kChunks + 2 * st + (lane >> 1)) * 64, fb);
       }
       return true;
     };
@@ -302,12 +323,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (row0 >= hi) break;
         bool vld;
         const int pg = page_of(p, b, row0, &vld);
-        for (int bb = 0; bb < 2; ++bb) {
-          uint32_t dst, fb;
-          if (!take(ring, dst, fb)) return false;
-          if (lane == 0)
-            tma_load_2d_pair(dst, &tm_cache2, 0, (pg * kChunks + (256 * bb + 128 * (int)rank) / 64) * 64, fb);
-        }
+        uint32_t dst, fb;
+        if (!take(ring, 2 * kChunkBytes, dst, fb)) return false;
+        if (lane < 2)
+          tma_load_2d_pair(dst + lane * kChunkBytes, &tm_cache2, 0,
+                           (pg * kChunks + (256 * lane + 128 * (int)rank) / 64) * 64, fb);
       }
       return true;
     };
@@ -333,14 +353,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           tc_fence_after();
         }
         const uint32_t d = tmem + (sb ? kColS1 : kColS0);
-        for (int c = 0; c < kChunks; ++c) {
+        for (int st = 0; st < kSStages; ++st) {
           uint32_t a0, empty;
           if (!ready(ring, a0, empty)) return false;
+          const int nc = st < kSStages - 1 ? 2 : 1;
+          for (int cc = 0; cc < nc; ++cc) {
+            const int c = 2 * st + cc;
 #pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t ad = smem_desc_sw128(a0 + ks * 32, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(s_q + c * LY::kQChunk + ks * 32, 16, 1024);
-            mma_pair_f16(d, ad, bd, idS, (c | ks) != 0);
+            for (int ks = 0; ks < 4; ++ks) {
+              const uint64_t ad = smem_desc_sw128(a0 + cc * kChunkBytes + ks * 32, 16, 1024);
+              const uint64_t bd = smem_desc_sw128(s_q + c * LY::kQChunk + ks * 32, 16, 1024);
+              mma_pair_f16(d, ad, bd, idS, (c | ks) != 0);
+            }
           }
           mma_commit_pair(empty, 0x3);
         }
@@ -351,18 +375,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (!mbar_wait(bar(B::p_full), j & 1, abort_flag)) return false;
         tc_fence_after();
         for (int pg_i = 0; pg_i < 4; ++pg_i) {
-          if (lo + kTile * j + 64 * pg_i >= hi) break;
-          for (int bb = 0; bb < 2; ++bb) {
+          // P^T chunk pg_i of tile j lives in slot (4j + pg_i) mod kPSlots; its
+          // release is committed even for pages past the end of the split
+          const int pslot = (4 * j + pg_i) % LY::kPSlots;
+          if (lo + kTile * j + 64 * pg_i < hi) {
             uint32_t a0, empty;
             if (!ready(ring, a0, empty)) return false;
+            for (int bb = 0; bb < 2; ++bb) {
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-              const uint64_t ad = smem_desc_sw128(a0 + ks * 2048, kBoxBytes, 1024);
-              const uint64_t bd = smem_desc_sw128(s_p + pg_i * LY::kPChunk + ks * 32, 16, 1024);
-              mma_pair_f16(tmem + kColO + bb * 128, ad, bd, idO, (j | pg_i | ks) != 0);
+              for (int ks = 0; ks < 4; ++ks) {
+                const uint64_t ad = smem_desc_sw128(a0 + bb * kChunkBytes + ks * 2048, kBoxBytes, 1024);
+                const uint64_t bd = smem_desc_sw128(s_p + pslot * LY::kPChunk + ks * 32, 16, 1024);
+                mma_pair_f16(tmem + kColO + bb * 128, ad, bd, idO, (j | pg_i | ks) != 0);
+              }
             }
             mma_commit_pair(empty, 0x3);
           }
+          mma_commit_pair(bar(B::p_free + pslot), 0x3);
         }
         mma_commit_pair(bar(B::o_done), 0x3);
         return true;
@@ -375,36 +404,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    // ================= softmax (both CTAs, warps 2-9) =================
-    // Per tile:
-    //   A  load the tile's scores (thread = row, HPW heads) into registers and
-    //      release the S^T buffer; per-head max over the warp (redux), then
-    //      over the 4 warps of the group
-    //   -- warp 0 of the group exchanges maxima with the peer and sets the
-    //      new running max (and the rescale factors) in shared memory
-    //   B  P = 2^(u - m) written to P^T, running row sums updated
-    constexpr int C = HPW < 32 ? HPW : 32;
-    const int g = (warp - kWarpSoft0) >> 2;    // warpgroup: heads [g*HPW, (g+1)*HPW)
+    // ================= softmax (both CTAs, warps 2-17) =================
+    // Four warpgroups, each a quarter of the heads (HPG) for this CTA's 128
+    // rows of the tile (thread = row).  Per tile:
+    //   A  load the tile's scores into registers and release the S^T buffer;
+    //      per-head max over the warp (redux), then over the 4 warps of the group
+    //   -- warp 0 of the group exchanges maxima with the peer's group of the
+    //      same heads and sets the new running max (and the rescale factors)
+    //   B  P = 2^(u - m) written to the P^T operand of the CTA that owns
+    //      these heads (CTA g/2), running row sums updated
+    constexpr int HPG = LY::HPG;
+    constexpr int C = HPG < 32 ? HPG : 32;
+    const int g = (warp - kWarpSoft0) >> 2;    // warpgroup: heads [g*HPG, (g+1)*HPG)
     const int q = warp & 3;                    // TMEM lane quadrant
     const int tok = 32 * q + lane;             // row within this CTA's half of the tile
     const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
-    const uint32_t p_dst = (g == (int)rank) ? s_p : mapa(s_p, (uint32_t)g);
-    const bool p_remote = g != (int)rank;
-    float* red_g = red + g * 4 * HPW;
+    const int owner = g >> 1;                  // CTA whose P^T holds these heads
+    const uint32_t p_dst = (owner == (int)rank) ? s_p : mapa(s_p, (uint32_t)owner);
+    const bool p_remote = owner != (int)rank;
+    const int hr0 = (g & 1) * HPG;             // first P^T row of these heads in the owner
+    float* red_g = red + g * 4 * HPG;
     float* alpha = own_max;                    // reused after the tile max is consumed
-    volatile int* changed_flag = reinterpret_cast<volatile int*>(misc + LY::kTmemSlot + 8) + g;
+    volatile int* changed_flag = reinterpret_cast<volatile int*>(misc + LY::kChanged) + g;
     // running row sums of this warp's 32 rows: chunk k, head C*k + lane % C
-    float l_acc[HPW / C];
+    float l_acc[HPG / C];
 #pragma unroll
-    for (int k = 0; k < HPW / C; ++k) l_acc[k] = 0.f;
+    for (int k = 0; k < HPG / C; ++k) l_acc[k] = 0.f;
     const int kt = 128 * (int)rank + tok;      // row within the pair tile
     const int ke = kt & ~1;
     const int wcol = ke & 63;
-    const uint32_t row_base = (ke >> 6) * LY::kPChunk + (wcol & 7) * 2;
+    const int pchunk = ke >> 6;                // P^T chunk (64 rows of the tile) this warp writes
     bool ok = true;
     for (int i = 0; i < n_tiles; ++i) {
       const int sb = i & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(B::s_full + sb), (i >> 1) & 1, abort_flag));
+      ok = __all_sync(0xffffffffu, mbar_wait<false>(bar(B::s_full + sb), (i >> 1) & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
       const int row = lo + kTile * i + kt;
@@ -416,43 +449,43 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       const float sl = vld ? p.scale_log2 : 0.f;
       // ---- A: scores into registers, release the buffer, per-head tile max
-      float u[HPW];
+      float u[HPG];
       {
-        const uint32_t sc = tmem + lane_addr + (sb ? kColS1 : kColS0) + g * HPW;
+        const uint32_t sc = tmem + lane_addr + (sb ? kColS1 : kColS0) + g * HPG;
 #pragma unroll
-        for (int k = 0; k < HPW / C; ++k) tmem_ld<C>(sc + C * k, u + C * k);
+        for (int k = 0; k < HPG / C; ++k) tmem_ld<C>(sc + C * k, u + C * k);
         tmem_wait_ld();
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(mapa(bar(B::s_free + sb), 0));
 #pragma unroll
-      for (int h = 0; h < HPW; ++h) {
+      for (int h = 0; h < HPG; ++h) {
         u[h] = vld ? u[h] * sl : -INFINITY;
         const float mx = redux_max(u[h]);
-        if (lane == (h & 31)) red_g[q * HPW + h] = mx;
+        if (lane == (h & 31)) red_g[q * HPG + h] = mx;
       }
       named_barrier(1 + g, 128);
       const int xb = i & 1;
-      const float* m_prev = m_used + ((i + 1) & 1) * NH + g * HPW;
-      float* m_next = m_used + (i & 1) * NH + g * HPW;
+      const float* m_prev = m_used + ((i + 1) & 1) * NH + g * HPG;
+      float* m_next = m_used + (i & 1) * NH + g * HPG;
       if (q == 0) {
-        for (int h = lane; h < HPW; h += 32) {
-          const float tm = fmaxf(fmaxf(red_g[h], red_g[HPW + h]), fmaxf(red_g[2 * HPW + h], red_g[3 * HPW + h]));
-          own_max[g * HPW + h] = tm;
-          st_cluster_f32(mapa(smem_u32(x_max + xb * NH + g * HPW + h), peer), tm);
+        for (int h = lane; h < HPG; h += 32) {
+          const float tm = fmaxf(fmaxf(red_g[h], red_g[HPG + h]), fmaxf(red_g[2 * HPG + h], red_g[3 * HPG + h]));
+          own_max[g * HPG + h] = tm;
+          st_cluster_f32(mapa(smem_u32(x_max + xb * NH + g * HPG + h), peer), tm);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(mapa(bar(B::mx_full + xb), peer));
         if (__all_sync(0xffffffffu, mbar_wait(bar(B::mx_full + xb), (i >> 1) & 1, abort_flag))) {
           int ch = 0;
-          for (int h = lane; h < HPW; h += 32) {
-            const float mt = fmaxf(own_max[g * HPW + h], x_max[xb * NH + g * HPW + h]);
+          for (int h = lane; h < HPG; h += 32) {
+            const float mt = fmaxf(own_max[g * HPG + h], x_max[xb * NH + g * HPG + h]);
             const float mo = m_prev[h];
             const float mn = (mt > mo + kRescaleLog2) ? mt : mo;
             m_next[h] = mn;
             // rescale factor for sums and accumulator kept so far (0 when nothing was kept)
-            alpha[g * HPW + h] = (mo == -INFINITY) ? 0.f : exp2_approx(mo - mn);
+            alpha[g * HPG + h] = (mo == -INFINITY) ? 0.f : exp2_approx(mo - mn);
             ch |= (mn != mo);
           }
           ch = __any_sync(0xffffffffu, ch);
@@ -464,27 +497,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const bool changed = *changed_flag != 0;
       // ---- B1: probabilities (fp32, in registers)
 #pragma unroll
-      for (int h = 0; h < HPW; ++h) {
+      for (int h = 0; h < HPG; ++h) {
         const float mn = m_next[h];
         u[h] = exp2_approx(u[h] - (mn == -INFINITY ? 0.f : mn));
       }
-      // the previous tile's O^T MMAs must be done: P^T buffer reuse and rescale
-      if (i >= 1) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(B::o_done), (i - 1) & 1, abort_flag));
+      // this warp's P^T chunk slot must have been released by the O^T MMAs
+      // of its previous use (1 or 2 tiles back); a moved running max also
+      // needs all of the previous tile's O^T MMAs done before the rescale
+      const int pn = 4 * i + pchunk;
+      const int pslot = pn % LY::kPSlots;
+      if (pn >= LY::kPSlots) {
+        ok = __all_sync(0xffffffffu,
+                        mbar_wait<false>(bar(B::p_free + pslot), ((pn / LY::kPSlots) - 1) & 1, abort_flag));
+        if (!ok) break;
+      }
+      const uint32_t row_base = pslot * LY::kPChunk + (wcol & 7) * 2;
+      if (i >= 1 && changed) {
+        ok = __all_sync(0xffffffffu, mbar_wait<false>(bar(B::o_done), (i - 1) & 1, abort_flag));
         if (!ok) break;
         tc_fence_after();
-        if (changed) {
+        {
           constexpr int CC = C < 16 ? C : 16;
 #pragma unroll 1
           for (int bb = 0; bb < 2; ++bb) {
 #pragma unroll 1
-            for (int k = 0; k < HPW / CC; ++k) {
-              const uint32_t oc = tmem + lane_addr + kColO + bb * 128 + g * HPW + CC * k;
+            for (int k = 0; k < HPG / CC; ++k) {
+              const uint32_t oc = tmem + lane_addr + kColO + bb * 128 + g * HPG + CC * k;
               float o[CC];
               tmem_ld<CC>(oc, o);
               tmem_wait_ld();
 #pragma unroll
-              for (int h = 0; h < CC; ++h) o[h] *= alpha[g * HPW + CC * k + h];
+              for (int h = 0; h < CC; ++h) o[h] *= alpha[g * HPG + CC * k + h];
               tmem_st<CC>(oc, o);
             }
           }
@@ -493,13 +536,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       // ---- B2: P^T (bf16, pairs of rows per 32-bit store), running row sums
 #pragma unroll
-      for (int k = 0; k < HPW / C; ++k) {
+      for (int k = 0; k < HPG / C; ++k) {
         float* uk = u + C * k;
 #pragma unroll
         for (int h = 0; h < C; h += 2) {
           const float send = (lane & 1) ? uk[h] : uk[h + 1];
           const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
-          const int hr = C * k + ((lane & 1) ? h + 1 : h);
+          const int hr = hr0 + C * k + ((lane & 1) ? h + 1 : h);
           __nv_bfloat162 pk = (lane & 1) ? __floats2bfloat162_rn(recv, uk[h + 1]) : __floats2bfloat162_rn(uk[h], recv);
           const uint32_t val = *reinterpret_cast<uint32_t*>(&pk);
           const uint32_t off = row_base + hr * 128 + ((((wcol >> 3) ^ (hr & 7))) << 4);
@@ -507,7 +550,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           else asm volatile("st.shared.b32 [%0], %1;" ::"r"(p_dst + off), "r"(val) : "memory");
         }
         const float ls = transpose_reduce<C>(uk, lane);
-        l_acc[k] = changed ? fmaf(l_acc[k], alpha[g * HPW + C * k + (lane % C)], ls) : l_acc[k] + ls;
+        l_acc[k] = changed ? fmaf(l_acc[k], alpha[g * HPG + C * k + (lane % C)], ls) : l_acc[k] + ls;
       }
       tc_fence_before();
       fence_proxy_async_cluster();
@@ -515,26 +558,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive_cluster(mapa(bar(B::p_full), 0));
     }
     // ---- epilogue: normalise O^T by the row sums, write o_part and lse
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(B::o_done), (n_tiles - 1) & 1, abort_flag));
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait<false>(bar(B::o_done), (n_tiles - 1) & 1, abort_flag));
     if (ok) {
       tc_fence_after();
 #pragma unroll
-      for (int k = 0; k < HPW / C; ++k)
-        if (lane < C) red_g[q * HPW + C * k + lane] = l_acc[k];
+      for (int k = 0; k < HPG / C; ++k)
+        if (lane < C) red_g[q * HPG + C * k + lane] = l_acc[k];
       named_barrier(1 + g, 128);
       float* inv_l = own_max;
       if (q == 0) {
-        for (int h = lane; h < HPW; h += 32) {
-          const float lt = red_g[h] + red_g[HPW + h] + red_g[2 * HPW + h] + red_g[3 * HPW + h];
-          l_own[g * HPW + h] = lt;
-          st_cluster_f32(mapa(smem_u32(l_x + g * HPW + h), peer), lt);
+        for (int h = lane; h < HPG; h += 32) {
+          const float lt = red_g[h] + red_g[HPG + h] + red_g[2 * HPG + h] + red_g[3 * HPG + h];
+          l_own[g * HPG + h] = lt;
+          st_cluster_f32(mapa(smem_u32(l_x + g * HPG + h), peer), lt);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(mapa(bar(B::l_full), peer));
         if (__all_sync(0xffffffffu, mbar_wait(bar(B::l_full), 0, abort_flag))) {
-          const float* m_fin = m_used + ((n_tiles - 1) & 1) * NH + g * HPW;
-          for (int h = lane; h < HPW; h += 32) {
-            const int hg = g * HPW + h;
+          const float* m_fin = m_used + ((n_tiles - 1) & 1) * NH + g * HPG;
+          for (int h = lane; h < HPG; h += 32) {
+            const int hg = g * HPG + h;
             const float lt = l_own[hg] + l_x[hg];
             inv_l[hg] = lt > 0.f ? 1.0f / lt : 0.f;
             if (leader && hg < p.n_heads)
@@ -550,8 +593,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int bb = 0; bb < 2; ++bb) {
           const int d = 256 * bb + 128 * (int)rank + tok;
 #pragma unroll 1
-          for (int k = 0; k < HPW / C; ++k) {
-            const int h0 = g * HPW + C * k;
+          for (int k = 0; k < HPG / C; ++k) {
+            const int h0 = g * HPG + C * k;
             float* op = p.o_part + ((size_t)r * p.n_heads * S + s) * MLA_D_C + d + (size_t)h0 * hstride;
             float o[C];
             tmem_ld<C>(tmem + lane_addr + kColO + bb * 128 + h0, o);

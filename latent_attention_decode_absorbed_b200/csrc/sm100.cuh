@@ -211,6 +211,7 @@ __device__ __forceinline__ void tmem_ld(uint32_t taddr, float* v);
                  : "r"(taddr));                                                             \
   }
 
+MLA_TMEM_LD_BODY(4, "{%0,%1,%2,%3}", "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]))
 MLA_TMEM_LD_BODY(8, "{%0,%1,%2,%3,%4,%5,%6,%7}", "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]),
                  "=r"(u[5]), "=r"(u[6]), "=r"(u[7]))
 MLA_TMEM_LD_BODY(16, "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}", "=r"(u[0]), "=r"(u[1]),
@@ -238,6 +239,7 @@ __device__ __forceinline__ void tmem_st(uint32_t taddr, const float* v);
                  : "memory");                                                               \
   }
 
+MLA_TMEM_ST_BODY(4, "{%1,%2,%3,%4}", "r"(u[0]), "r"(u[1]), "r"(u[2]), "r"(u[3]))
 MLA_TMEM_ST_BODY(8, "{%1,%2,%3,%4,%5,%6,%7,%8}", "r"(u[0]), "r"(u[1]), "r"(u[2]), "r"(u[3]), "r"(u[4]),
                  "r"(u[5]), "r"(u[6]), "r"(u[7]))
 MLA_TMEM_ST_BODY(16, "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16}", "r"(u[0]), "r"(u[1]),
