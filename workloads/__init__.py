@@ -79,9 +79,15 @@ def _rng(seed: int, tensor: int, index: int = 0) -> np.random.Generator:
 def round_bf16(x: np.ndarray) -> np.ndarray:
     """Round float32 values to the nearest bfloat16 (ties to even); returns
     float32 holding bf16-representable values.  Storage cast of an input."""
-    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
-    u = (u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000
-    return u.astype(np.uint32).view(np.float32)
+    u = np.array(x, dtype=np.float32, copy=True).view(np.uint32)
+    if not np.isfinite(u.view(np.float32)).all():
+        raise ValueError("round_bf16: non-finite input")
+    # finite inputs: u + 0x8000 stays below 2**32, so 32-bit arithmetic is exact
+    lsb = (u >> 16) & 1
+    u += np.uint32(0x7FFF)
+    u += lsb
+    u &= np.uint32(0xFFFF0000)
+    return u.view(np.float32)
 
 
 def bf16_bits(x: np.ndarray) -> np.ndarray:
