@@ -70,6 +70,26 @@ def recorded_traffic(workload):
     return None
 
 
+def max_over_ranks(values, world, device=None):
+    """Element-wise max of per-rank timings (list of floats) over all ranks.
+
+    Multi-GPU numbers are the slowest rank's: every rank times the same K
+    steps between barriers, and the job is done when the last one is."""
+    if world <= 1:
+        return list(values)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_throughput(world, tokens_per_step, steps, elapsed_ms):
+    """Whole-job tokens/s: every rank completes `tokens_per_step` query tokens
+    per step (independent sequences per GPU, weak scaling)."""
+    return world * tokens_per_step * steps / (elapsed_ms / 1e3)
+
+
 def algorithmic(w, lens):
     rows = int(lens.sum())
     bytes_ = rows * CACHE_BYTES[w.cache_dtype]
@@ -294,15 +314,12 @@ def run_gpu(args, w, rank, world, local_rank):
     assert int(step.err.item()) == 0, "device error flag set"
 
     # max over ranks
-    t = torch.tensor([elapsed_ms, e2e_ms, float(np.mean(decode_ms))], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    elapsed_ms, e2e_ms, dec_ms = t.tolist()
+    elapsed_ms, e2e_ms, dec_ms = max_over_ranks([elapsed_ms, e2e_ms, float(np.mean(decode_ms))], world, dev)
     if rank != 0:
         return 0
     tokens_per_step = w.batch * w.q_len
-    value = world * tokens_per_step * args.steps / (elapsed_ms / 1e3)
-    e2e_value = world * tokens_per_step * args.steps / (e2e_ms / 1e3)
+    value = job_throughput(world, tokens_per_step, args.steps, elapsed_ms)
+    e2e_value = job_throughput(world, tokens_per_step, args.steps, e2e_ms)
     pk = peaks()
     achieved = alg_bytes / (dec_ms / 1e3) / 1e9
     traffic = recorded_traffic(w.name)

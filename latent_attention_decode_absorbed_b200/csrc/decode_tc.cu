@@ -32,8 +32,8 @@
 // (leader CTA only), 2-9 softmax (two warpgroups, one per half of the heads;
 // thread = cached row).
 //
-// Softmax per tile: each warp takes the per-head max of its 32 rows with
-// redux.sync, the 4 warps of a warpgroup combine through shared memory, the
+// Softmax per tile: each warp takes the per-head max of its 32 rows with a
+// shuffle butterfly, the 4 warps of a warpgroup combine through shared memory, the
 // pair exchanges its maxima through distributed shared memory, and the
 // running max only moves when the tile max exceeds it by more than 2^8 (the
 // accumulator is rescaled in TMEM then).  P = 2^(u - m) is written as bf16
@@ -52,18 +52,26 @@ namespace {
 using namespace sm100;
 
 constexpr int kSoftGroups = 4;           // softmax warpgroups, each a quarter of the heads
-constexpr int kThreads = 32 * (2 + 4 * kSoftGroups);  // 18 warps: see the role map above
+// 18 warps (bf16 cache) or 20 (e4m3 cache: two converter warps): see the role map above
+template <bool F8>
+constexpr int kThreadsT = 32 * ((F8 ? 4 : 2) + 4 * kSoftGroups);
+constexpr int kWarpConv0 = 2, kConvWarps = 2;  // e4m3 converters
+constexpr int kBox8 = 4096;                    // one e4m3 block: 64 rows x 64 bytes
+constexpr int kStage8 = 4 * kBox8;             // e4m3 staging of one stage (at most four blocks)
 constexpr int kSlotBytes = 32768;         // one ring stage
 constexpr int kBoxBytes = 8192;           // 64 rows x 128 bytes
 constexpr int kChunkBytes = 16384;        // one column chunk of 128 rows (both pages)
 constexpr int kSStages = 5;               // score stages per tile: chunks {0,1} {2,3} {4,5} {6,7} {8}
+constexpr bool kL2Hints = true;           // L2 residency policies on the cache loads
 
 constexpr int kTile = 256;                // cached rows per pair tile
 constexpr int kChunks = 9;                // 576 / 64 column chunks
 constexpr float kRescaleLog2 = 8.0f;      // lazy rescale threshold (log2 units)
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
-constexpr int kWarpProd = 0, kWarpMma = 1, kWarpSoft0 = 2;
+constexpr int kWarpProd = 0, kWarpMma = 1;
+template <bool F8>
+constexpr int kWarpSoft0T = F8 ? 4 : 2;
 
 struct TcParams {
   int n_heads, q_len, batch;
@@ -72,12 +80,13 @@ struct TcParams {
   const int32_t* seq_lens;
   int num_splits, split_tokens;
   float scale_log2;            // softmax_scale * log2(e)
+  const float* cache_scale;    // e4m3 cache: per-row dequantisation scale [num_pages * 64]
   float* o_part;
   float* lse_part;
   int32_t* err;
 };
 
-template <int NH>
+template <int NH, bool F8>
 struct Layout {
   static constexpr int HPW = NH / 2;                      // heads per CTA (its half of Q and P^T)
   static constexpr int HPG = NH / kSoftGroups;            // heads per softmax warpgroup
@@ -98,10 +107,13 @@ struct Layout {
   static constexpr int kMiscBytes = kLX + NH * 4;
   // ring of operand stages: as many as fit next to Q, P^T and the misc area (at most 6)
   static constexpr int kFixed = kChunks * kQChunk + kPSlots * kPChunk + kMiscBytes + 1024;
-  static constexpr int kFit = (227 * 1024 - kFixed) / kSlotBytes;
+  // (e4m3 cache: each stage also has a staging slot for the raw codes)
+  static constexpr int kPerSlot = kSlotBytes + (F8 ? kStage8 : 0);
+  static constexpr int kFit = (227 * 1024 - kFixed) / kPerSlot;
   static constexpr int kSlots = kFit > 6 ? 6 : kFit;
   static constexpr int kRing = 0;
-  static constexpr int kQ = kRing + kSlots * kSlotBytes;
+  static constexpr int kStaging = kRing + kSlots * kSlotBytes;
+  static constexpr int kQ = kStaging + (F8 ? kSlots * kStage8 : 0);
   static constexpr int kP = kQ + kChunks * kQChunk;
   static constexpr int kMisc = kP + kPSlots * kPChunk;
   static constexpr int kSmem = kMisc + kMiscBytes + 1024;  // + alignment slack
@@ -122,13 +134,12 @@ struct Bars {
   static constexpr int q_full = base + 8;            //       leader: Q of both CTAs loaded
   static constexpr int l_full = base + 9;            //       both: the peer's row sums arrived
   static constexpr int p_free = base + 10;           // [6]   both: O^T MMAs done with a P^T chunk slot
+  // e4m3 cache only
+  static constexpr int q_ready = base + 16;          //       leader: both CTAs converted Q to f16
+  static constexpr int sfull8 = base + 17;           // [NS]  local: TMA bytes of a staging slot
+  static constexpr int sempty8 = base + 17 + NS;     // [NS]  local: converters done with the staging slot
+  static constexpr int end = base + 17 + 2 * NS;
 };
-
-__device__ __forceinline__ float redux_max(float v) {
-  float r;
-  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
-  return r;
-}
 
 // Sum over the 32 lanes of a warp of each of C per-lane values, returned
 // transposed: lane l gets the sum of index l % C.  log2(32) shuffle stages;
@@ -149,6 +160,28 @@ __device__ __forceinline__ float transpose_reduce(float* v, int lane) {
       const float keep = up ? v[j + off] : v[j];
       const float send = up ? v[j] : v[j + off];
       v[j] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+  }
+  return v[0];
+}
+
+// Max over the 32 lanes of each of C per-lane values, returned transposed
+// like transpose_reduce (lane l gets the max of index l % C); v is clobbered.
+template <int C>
+__device__ __forceinline__ float transpose_max(float* v, int lane) {
+#pragma unroll
+  for (int off = 16; off >= C; off >>= 1) {
+#pragma unroll
+    for (int j = 0; j < C; ++j) v[j] = fmaxf(v[j], __shfl_xor_sync(0xffffffffu, v[j], off));
+  }
+#pragma unroll
+  for (int off = C / 2; off >= 1; off >>= 1) {
+    const bool up = (lane & off) != 0;
+#pragma unroll
+    for (int j = 0; j < off; ++j) {
+      const float keep = up ? v[j + off] : v[j];
+      const float send = up ? v[j] : v[j + off];
+      v[j] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, off));
     }
   }
   return v[0];
@@ -182,14 +215,16 @@ struct Ring {
   uint32_t kc = 0;
 };
 
-template <int NH>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+template <int NH, bool F8>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_constant__ CUtensorMap tm_cache2,
                      const __grid_constant__ CUtensorMap tm_q, const TcParams p) {
-  using LY = Layout<NH>;
+  using LY = Layout<NH, F8>;
   constexpr int HPW = LY::HPW;
+  constexpr int kThreads = kThreadsT<F8>;
+  constexpr int kWarpSoft0 = kWarpSoft0T<F8>;
   using B = Bars<LY::kSlots>;
-  static_assert(B::base + 16 <= 64, "barrier area");
+  static_assert(B::end <= 64, "barrier area");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -226,9 +261,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   // ---- set-up: barriers, TMEM, cluster sync
   if (threadIdx.x == 0) {
     for (int i = 0; i < LY::kSlots; ++i) {
-      mbar_init(bar(B::full + i), 1);
+      // bf16: one expect-tx arrival (the leader's producer) plus both CTAs' bytes;
+      // e4m3: one arrival per converter warp of both CTAs
+      mbar_init(bar(B::full + i), F8 ? 2 * kConvWarps : 1);
       mbar_init(bar(B::empty + i), 1);
+      if constexpr (F8) {
+        mbar_init(bar(B::sfull8 + i), 1);
+        mbar_init(bar(B::sempty8 + i), kConvWarps);
+      }
     }
+    if constexpr (F8) mbar_init(bar(B::q_ready), 2 * kConvWarps);
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(B::s_full + i), 1);
       mbar_init(bar(B::s_free + i), 2 * 4 * kSoftGroups);
@@ -271,7 +313,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   auto ready = [&](Ring& rg, uint32_t& src, uint32_t& empty) -> bool {
     const uint32_t slot = rg.kc % rg.slots;
     const uint32_t ph = (rg.kc / rg.slots) & 1u;
-    if (!mbar_wait<false>(rg.full0 + 8 * slot, ph, abort_flag)) return false;
+    // e4m3: the converters arrive after generic-proxy writes (cluster scope)
+    if (!mbar_wait<F8>(rg.full0 + 8 * slot, ph, abort_flag)) return false;
     tc_fence_after();
     src = rg.base + slot * kSlotBytes;
     empty = rg.empty0 + 8 * slot;
@@ -285,6 +328,168 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if ((h & 1) != (int)rank) continue;
       p.o_part[(((size_t)r * p.n_heads + h) * S + s) * MLA_D_C + d] = 0.f;
       if (d == 0) p.lse_part[((size_t)r * p.n_heads + h) * S + s] = -INFINITY;
+    }
+  } else if (F8 && warp == kWarpProd) {
+    // ============ TMA producer, e4m3 cache (both CTAs) ============
+    // The same stages in the same order as the bf16 producer, but each CTA
+    // loads raw e4m3 blocks ([64 rows x 64 bytes], one per lane) into its own
+    // staging slot and local barrier; the converter warps widen them into the
+    // operand ring.  Staging block b of a stage lands at b * 4 KB and is
+    // widened to b * 8 KB: score stages use b = 2 * chunk + page, value
+    // stages b = 2 * dims block + half.
+    if constexpr (F8) {
+      uint32_t kc = 0;
+      auto take8 = [&](uint32_t nbox, uint32_t& dst, uint32_t& fb) -> bool {
+        const uint32_t slot = kc % LY::kSlots;
+        const uint32_t ph = (kc / LY::kSlots) & 1u;
+        bool ok = true;
+        if (lane == 0) {
+          ok = mbar_wait<false>(bar(B::sempty8 + slot), ph ^ 1u, abort_flag);
+          if (ok) mbar_arrive_expect_tx(bar(B::sfull8 + slot), nbox * kBox8);
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        dst = s_base + LY::kStaging + slot * kStage8;
+        fb = bar(B::sfull8 + slot);
+        ++kc;
+        return ok;
+      };
+      if (lane == 0) {
+        tma_prefetch_desc(&tm_cache);
+        tma_prefetch_desc(&tm_q);
+        mbar_arrive_expect_tx(bar(B::q_full), kChunks * LY::kQChunk);
+        for (int c = 0; c < kChunks; ++c)
+          tma_load_3d(s_q + c * LY::kQChunk, &tm_q, 64 * c, (int)rank * HPW, r, bar(B::q_full));
+      }
+      auto load_s8 = [&](int i) -> bool {
+        bool vv;
+        const int pg = page_of(p, b, lo + kTile * i + 128 * (int)rank + 64 * (lane & 1), &vv);
+        for (int st = 0; st < kSStages; ++st) {
+          const int nc = st < kSStages - 1 ? 2 : 1;
+          uint32_t dst, fb;
+          if (!take8(2 * nc, dst, fb)) return false;
+          if (lane < 2 * nc) tma_load_2d(dst + lane * kBox8, &tm_cache, 0, (pg * kChunks + 2 * st + (lane >> 1)) * 64, fb);
+        }
+        return true;
+      };
+      auto load_o8 = [&](int j) -> bool {
+        for (int pg_i = 0; pg_i < 4; ++pg_i) {
+          const int row0 = lo + kTile * j + 64 * pg_i;
+          if (row0 >= hi) break;
+          bool vld;
+          const int pg = page_of(p, b, row0, &vld);
+          uint32_t dst, fb;
+          if (!take8(4, dst, fb)) return false;
+          if (lane < 4) {
+            const int blk = (256 * (lane >> 1) + 128 * (int)rank) / 64 + (lane & 1);
+            tma_load_2d(dst + lane * kBox8, &tm_cache, 0, (pg * kChunks + blk) * 64, fb);
+          }
+        }
+        return true;
+      };
+      bool ok = load_s8(0);
+      if (ok && n_tiles > 1) ok = load_s8(1);
+      for (int i = 0; i < n_tiles && ok; ++i) {
+        if (i + 2 < n_tiles) ok = load_s8(i + 2);
+        if (ok) ok = load_o8(i);
+      }
+    }
+  } else if (F8 && warp >= kWarpConv0 && warp < kWarpConv0 + kConvWarps) {
+    // ============ e4m3 -> f16 converters (both CTAs) ============
+    // First Q (bf16 -> f16 in place, once per unit), then every stage in the
+    // MMA's order: wait for the staging slot's bytes and the operand slot's
+    // release, widen the codes exactly (e4m3 values are f16 values), write
+    // them 128-byte swizzled, make them visible to the tensor core and arrive
+    // on the leader's full barrier.  Value stages are also multiplied by the
+    // row's dequantisation scale (one f16 rounding: the dequantised value);
+    // for scores the softmax applies the scale to the row's dot products.
+    if constexpr (F8) {
+      const int ct = threadIdx.x - 32 * kWarpConv0;
+      constexpr int kCT = 32 * kConvWarps;
+      bool ok = __all_sync(0xffffffffu, mbar_wait<false>(bar(B::q_full), 0, abort_flag));
+      if (ok) {
+        for (int i = ct; i < kChunks * LY::kQChunk / 16; i += kCT) {
+          uint4 v = *reinterpret_cast<const uint4*>(smem + LY::kQ + 16 * i);
+          uint32_t* w = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+            const __half2 h = __floats2half2_rn(f.x, f.y);
+            w[e] = *reinterpret_cast<const uint32_t*>(&h);
+          }
+          *reinterpret_cast<uint4*>(smem + LY::kQ + 16 * i) = v;
+        }
+        fence_proxy_async_cluster();     // read by the pair's MMAs
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(mapa(bar(B::q_ready), 0));
+      }
+      uint32_t kc = 0;
+      auto convert = [&](int nbox, int scale_page) -> bool {
+        // scale_page >= 0: value stage of that page (lane l holds rows l, l + 32)
+        float s_lo = 1.f, s_hi = 1.f;
+        if (scale_page >= 0) {
+          s_lo = p.cache_scale[(size_t)scale_page * 64 + lane];
+          s_hi = p.cache_scale[(size_t)scale_page * 64 + 32 + lane];
+        }
+        const uint32_t slot = kc % LY::kSlots;
+        const uint32_t ph = (kc / LY::kSlots) & 1u;
+        ++kc;
+        if (!__all_sync(0xffffffffu, mbar_wait<false>(bar(B::sfull8 + slot), ph, abort_flag))) return false;
+        if (!__all_sync(0xffffffffu, mbar_wait<false>(bar(B::empty + slot), ph ^ 1u, abort_flag))) return false;
+        const uint8_t* src = smem + LY::kStaging + slot * kStage8;
+        uint8_t* dst = smem + LY::kRing + slot * kSlotBytes;
+        // 16 codes (one quarter of a 64-byte row) per step
+        for (int c = ct; c < nbox * 256; c += kCT) {
+          const int box = c >> 8, row = (c >> 2) & 63, qq = c & 3;
+          const uint4 codes = *reinterpret_cast<const uint4*>(src + box * kBox8 + row * 64 + qq * 16);
+          const uint32_t* cw = reinterpret_cast<const uint32_t*>(&codes);
+          const float sa = __shfl_sync(0xffffffffu, s_lo, row & 31);
+          const float sb = __shfl_sync(0xffffffffu, s_hi, row & 31);
+          const __half2 rs2 = __float2half2_rn(row < 32 ? sa : sb);
+          uint32_t hw[8];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+              const __half2_raw r2 = __nv_cvt_fp8x2_to_halfraw2(
+                  static_cast<__nv_fp8x2_storage_t>((cw[e] >> (16 * hf)) & 0xffffu), __NV_E4M3);
+              __half2 h2 = *reinterpret_cast<const __half2*>(&r2);
+              if (scale_page >= 0) h2 = __hmul2(h2, rs2);
+              hw[2 * e + hf] = *reinterpret_cast<const uint32_t*>(&h2);
+            }
+          }
+          uint8_t* rowp = dst + box * kBoxBytes + row * 128;
+          *reinterpret_cast<uint4*>(rowp + (((2 * qq) ^ (row & 7)) << 4)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+          *reinterpret_cast<uint4*>(rowp + (((2 * qq + 1) ^ (row & 7)) << 4)) = make_uint4(hw[4], hw[5], hw[6], hw[7]);
+        }
+        fence_proxy_async_cluster();     // read by the pair's MMAs
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive_local(bar(B::sempty8 + slot));
+          mbar_arrive_cluster(mapa(bar(B::full + slot), 0));
+        }
+        return true;
+      };
+      auto conv_s = [&]() -> bool {
+        for (int st = 0; st < kSStages; ++st)
+          if (!convert(st < kSStages - 1 ? 4 : 2, -1)) return false;
+        return true;
+      };
+      auto conv_o = [&](int j) -> bool {
+        for (int pg_i = 0; pg_i < 4; ++pg_i) {
+          const int row0 = lo + kTile * j + 64 * pg_i;
+          if (row0 >= hi) break;
+          bool vld;
+          const int pg = page_of(p, b, row0, &vld);
+          if (!convert(4, pg)) return false;
+        }
+        return true;
+      };
+      if (ok) ok = conv_s();
+      if (ok && n_tiles > 1) ok = conv_s();
+      for (int i = 0; i < n_tiles && ok; ++i) {
+        if (i + 2 < n_tiles) ok = conv_s();
+        if (ok) ok = conv_o(i);
+      }
     }
   } else if (warp == kWarpProd) {
     // ============ TMA producer (both CTAs), in the order the MMA consumes ============
@@ -304,6 +509,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       for (int c = 0; c < kChunks; ++c)
         tma_load_3d_pair(s_q + c * LY::kQChunk, &tm_q, 64 * c, (int)rank * HPW, r, q_bar);
     }
+    // L2 residency: this CTA's score rows are re-read (by the peer and by
+    // itself) for the value operand two tiles later, so they are loaded
+    // evict-last; value loads are the rows' last use and go evict-first.
+    const uint64_t pol_keep = kL2Hints ? policy_evict_last() : 0;
+    const uint64_t pol_drop = kL2Hints ? policy_evict_first() : 0;
     auto load_s = [&](int i) -> bool {
       bool vv;
       const int pg = page_of(p, b, lo + kTile * i + 128 * (int)rank + 64 * (lane & 1), &vv);
@@ -311,9 +521,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int nc = st < kSStages - 1 ? 2 : 1;
         uint32_t dst, fb;
         if (!take(ring, nc * kChunkBytes, dst, fb)) return false;
-        if (lane < 2 * nc)
-          tma_load_2d_pair(dst + (lane >> 1) * kChunkBytes + (lane & 1) * kBoxBytes, &tm_cache, 0,
-                           (pg * kChunks + 2 * st + (lane >> 1)) * 64, fb);
+        if (lane < 2 * nc) {
+          const uint32_t d = dst + (lane >> 1) * kChunkBytes + (lane & 1) * kBoxBytes;
+          const int y = (pg * kChunks + 2 * st + (lane >> 1)) * 64;
+          if (kL2Hints) tma_load_2d_pair_hint(d, &tm_cache, 0, y, fb, pol_keep);
+          else tma_load_2d_pair(d, &tm_cache, 0, y, fb);
+        }
       }
       return true;
     };
@@ -325,9 +538,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int pg = page_of(p, b, row0, &vld);
         uint32_t dst, fb;
         if (!take(ring, 2 * kChunkBytes, dst, fb)) return false;
-        if (lane < 2)
-          tma_load_2d_pair(dst + lane * kChunkBytes, &tm_cache2, 0,
-                           (pg * kChunks + (256 * lane + 128 * (int)rank) / 64) * 64, fb);
+        if (lane < 2) {
+          const int y = (pg * kChunks + (256 * lane + 128 * (int)rank) / 64) * 64;
+          if (kL2Hints) tma_load_2d_pair_hint(dst + lane * kChunkBytes, &tm_cache2, 0, y, fb, pol_drop);
+          else tma_load_2d_pair(dst + lane * kChunkBytes, &tm_cache2, 0, y, fb);
+        }
       }
       return true;
     };
@@ -342,9 +557,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // order: S(0), S(1), then per tile i: S(i+2), O(i) -- the score GEMM runs
     // two tiles ahead so the softmax of tile i overlaps S(i+1), O(i-1), S(i+2)
     if (leader && lane == 0) {
-      constexpr uint32_t idS = idesc_f16(256, NH, false, false);
-      constexpr uint32_t idO = idesc_f16(256, NH, true, false);
-      bool ok = mbar_wait(bar(B::q_full), 0, abort_flag);
+      // e4m3 cache: the operands are f16 (widened codes, Q and P in f16)
+      constexpr uint32_t idS = idesc_f16(256, NH, false, false, F8);
+      constexpr uint32_t idO = idesc_f16(256, NH, true, false, F8);
+      bool ok = mbar_wait(bar(F8 ? B::q_ready : B::q_full), 0, abort_flag);
       tc_fence_after();
       auto issue_s = [&](int i) -> bool {
         const int sb = i & 1;
@@ -408,7 +624,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // Four warpgroups, each a quarter of the heads (HPG) for this CTA's 128
     // rows of the tile (thread = row).  Per tile:
     //   A  load the tile's scores into registers and release the S^T buffer;
-    //      per-head max over the warp (redux), then over the 4 warps of the group
+    //      per-head max over the warp (shuffle butterfly), then over the 4 warps of the group
     //   -- warp 0 of the group exchanges maxima with the peer's group of the
     //      same heads and sets the new running max (and the rescale factors)
     //   B  P = 2^(u - m) written to the P^T operand of the CTA that owns
@@ -442,12 +658,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const int row = lo + kTile * i + kt;
       bool vld = row < hi;
+      float rsc = 1.f;                         // e4m3: the row's dequantisation scale
       if (vld) {
         bool pok;
-        (void)page_of(p, b, row, &pok);
+        const int pg = page_of(p, b, row, &pok);
         if (!pok) { vld = false; flag_error(p.err, MLA_DEVERR_PAGE); }
+        else if constexpr (F8) rsc = p.cache_scale[(size_t)pg * 64 + (row & 63)];
       }
-      const float sl = vld ? p.scale_log2 : 0.f;
+      const float sl = vld ? p.scale_log2 * rsc : 0.f;
       // ---- A: scores into registers, release the buffer, per-head tile max
       float u[HPG];
       {
@@ -460,10 +678,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(mapa(bar(B::s_free + sb), 0));
 #pragma unroll
-      for (int h = 0; h < HPG; ++h) {
-        u[h] = vld ? u[h] * sl : -INFINITY;
-        const float mx = redux_max(u[h]);
-        if (lane == (h & 31)) red_g[q * HPG + h] = mx;
+      for (int h = 0; h < HPG; ++h) u[h] = vld ? u[h] * sl : -INFINITY;
+      {
+        // per-head max over the warp's 32 rows: a transposing butterfly
+        // leaves head C*k + lane%C's max in lane `lane`
+        float t[HPG];
+#pragma unroll
+        for (int h = 0; h < HPG; ++h) t[h] = u[h];
+#pragma unroll
+        for (int k = 0; k < HPG / C; ++k) {
+          const float mx = transpose_max<C>(t + C * k, lane);
+          if (lane < C) red_g[q * HPG + C * k + lane] = mx;
+        }
       }
       named_barrier(1 + g, 128);
       const int xb = i & 1;
@@ -502,8 +728,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         u[h] = exp2_approx(u[h] - (mn == -INFINITY ? 0.f : mn));
       }
       // this warp's P^T chunk slot must have been released by the O^T MMAs
-      // of its previous use (1 or 2 tiles back); a moved running max also
-      // needs all of the previous tile's O^T MMAs done before the rescale
+      // of its previous use (1 or 2 tiles back), and every phase of o_done is
+      // observed in order: a parity wait cannot tell a barrier two phases
+      // behind from one that is done, so skipping phases here would let the
+      // rescale and the epilogue read the accumulator before the last O^T
+      // MMAs complete
       const int pn = 4 * i + pchunk;
       const int pslot = pn % LY::kPSlots;
       if (pn >= LY::kPSlots) {
@@ -512,10 +741,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (!ok) break;
       }
       const uint32_t row_base = pslot * LY::kPChunk + (wcol & 7) * 2;
-      if (i >= 1 && changed) {
+      if (i >= 1) {
         ok = __all_sync(0xffffffffu, mbar_wait<false>(bar(B::o_done), (i - 1) & 1, abort_flag));
         if (!ok) break;
         tc_fence_after();
+      }
+      if (i >= 1 && changed) {
         {
           constexpr int CC = C < 16 ? C : 16;
 #pragma unroll 1
@@ -543,8 +774,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const float send = (lane & 1) ? uk[h] : uk[h + 1];
           const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
           const int hr = hr0 + C * k + ((lane & 1) ? h + 1 : h);
-          __nv_bfloat162 pk = (lane & 1) ? __floats2bfloat162_rn(recv, uk[h + 1]) : __floats2bfloat162_rn(uk[h], recv);
-          const uint32_t val = *reinterpret_cast<uint32_t*>(&pk);
+          const float mine = (lane & 1) ? uk[h + 1] : uk[h];
+          uint32_t val;
+          if constexpr (F8) {
+            const __half2 pk = (lane & 1) ? __floats2half2_rn(recv, mine) : __floats2half2_rn(mine, recv);
+            val = *reinterpret_cast<const uint32_t*>(&pk);
+          } else {
+            const __nv_bfloat162 pk = (lane & 1) ? __floats2bfloat162_rn(recv, mine) : __floats2bfloat162_rn(mine, recv);
+            val = *reinterpret_cast<const uint32_t*>(&pk);
+          }
           const uint32_t off = row_base + hr * 128 + ((((wcol >> 3) ^ (hr & 7))) << 4);
           if (p_remote) st_cluster_b32(p_dst + off, val);
           else asm volatile("st.shared.b32 [%0], %1;" ::"r"(p_dst + off), "r"(val) : "memory");
@@ -646,25 +884,25 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-template <int NH>
+template <int NH, bool F8>
 cudaError_t launch_nh(const DecodeArgs& a, const CUtensorMap& tc, const CUtensorMap& tc2, const CUtensorMap& tq,
                       cudaStream_t st) {
-  using LY = Layout<NH>;
-  cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<NH>, cudaFuncAttributeMaxDynamicSharedMemorySize, LY::kSmem);
+  using LY = Layout<NH, F8>;
+  cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<NH, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, LY::kSmem);
   if (e != cudaSuccess) return e;
   TcParams p{a.n_heads, a.q_len, a.batch, a.block_table, a.max_pages, a.num_pages, a.seq_lens, a.num_splits,
-             a.split_tokens, a.softmax_scale * 1.4426950408889634f, a.o_part, a.lse_part, a.err};
+             a.split_tokens, a.softmax_scale * 1.4426950408889634f, a.cache_scale, a.o_part, a.lse_part, a.err};
   const long long units = (long long)a.batch * a.q_len * a.num_splits;
   dim3 grid((unsigned)(2 * units));
-  decode_tc_kernel<NH><<<grid, kThreads, LY::kSmem, st>>>(tc, tc2, tq, p);
+  decode_tc_kernel<NH, F8><<<grid, kThreadsT<F8>, LY::kSmem, st>>>(tc, tc2, tq, p);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 bool decode_tc_supported(const DecodeArgs& a) {
-  return a.q_dtype == MLA_BF16 && a.cache_dtype == MLA_BF16 && a.page_size == 64 &&
-         (long long)a.batch * a.q_len * a.num_splits * 2 < (1ll << 31);
+  return a.q_dtype == MLA_BF16 && (a.cache_dtype == MLA_BF16 || a.cache_dtype == MLA_E4M3) &&
+         a.page_size == 64 && (long long)a.batch * a.q_len * a.num_splits * 2 < (1ll << 31);
 }
 
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st) {
@@ -673,9 +911,22 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st) {
   const int NH = a.n_heads <= 16 ? 16 : a.n_heads <= 32 ? 32 : a.n_heads <= 64 ? 64 : 128;
   const int HPW = NH / 2;
   CUtensorMap tc, tc2, tq;
-  // the page-blocked pool as 2-D [num_pages * 9 * 64 lines x 64 columns], 128-byte lines:
-  // boxes of 64 lines (one block) and of 128 lines (two adjacent blocks)
-  for (int k = 0; k < 2; ++k) {
+  const bool f8 = a.cache_dtype == MLA_E4M3;
+  // the page-blocked pool as 2-D [num_pages * 9 * 64 lines x 64 columns]:
+  // bf16, 128-byte lines: boxes of 64 lines (one block) and of 128 lines (two
+  // adjacent blocks); e4m3, 64-byte lines: boxes of one block, unswizzled
+  if (f8) {
+    cuuint64_t dims[2] = {64, (cuuint64_t)a.num_pages * kChunks * 64};
+    cuuint64_t strides[1] = {64};
+    cuuint32_t box[2] = {64, 64};
+    cuuint32_t es[2] = {1, 1};
+    if (enc(&tc, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(a.cache), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+    tc2 = tc;
+  }
+  for (int k = 0; k < 2 && !f8; ++k) {
     cuuint64_t dims[2] = {64, (cuuint64_t)a.num_pages * kChunks * 64};
     cuuint64_t strides[1] = {128};
     cuuint32_t box[2] = {64, k == 0 ? 64u : 128u};
@@ -695,11 +946,19 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
+  if (f8) {
+    switch (NH) {
+      case 16: return launch_nh<16, true>(a, tc, tc2, tq, st);
+      case 32: return launch_nh<32, true>(a, tc, tc2, tq, st);
+      case 64: return launch_nh<64, true>(a, tc, tc2, tq, st);
+      default: return launch_nh<128, true>(a, tc, tc2, tq, st);
+    }
+  }
   switch (NH) {
-    case 16: return launch_nh<16>(a, tc, tc2, tq, st);
-    case 32: return launch_nh<32>(a, tc, tc2, tq, st);
-    case 64: return launch_nh<64>(a, tc, tc2, tq, st);
-    default: return launch_nh<128>(a, tc, tc2, tq, st);
+    case 16: return launch_nh<16, false>(a, tc, tc2, tq, st);
+    case 32: return launch_nh<32, false>(a, tc, tc2, tq, st);
+    case 64: return launch_nh<64, false>(a, tc, tc2, tq, st);
+    default: return launch_nh<128, false>(a, tc, tc2, tq, st);
   }
 }
 

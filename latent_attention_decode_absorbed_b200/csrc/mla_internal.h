@@ -38,7 +38,7 @@ struct DecodeArgs {
   float* o_part; float* lse_part; int32_t* err;
 };
 cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t st);
-// tcgen05 path: bf16 queries over a bf16 cache
+// tcgen05 path: bf16 queries over a bf16 or e4m3 cache
 bool decode_tc_supported(const DecodeArgs& a);
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st);
 

@@ -207,6 +207,10 @@ CASES = [
     ("heads48_bf16", "bf16", [200, 513], 1, 48, 256),
     ("long_split_bf16", "bf16", [5000], 1, 128, 4096),
     ("ragged_e4m3", "e4m3", [5, 400, 1025], 2, 128, 256),
+    ("heads64_e4m3", "e4m3", [300, 70], 1, 64, 128),
+    ("heads16_many_splits_e4m3", "e4m3", [700], 1, 16, 64),
+    ("multi_tile_e4m3", "e4m3", [1100, 600], 2, 128, 1024),
+    ("long_split_e4m3", "e4m3", [5000], 1, 128, 4096),
     ("tiny_f32", "f32", [256, 37], 1, 16, 64),
 ]
 
