@@ -152,6 +152,8 @@ mla_status mla_cache_append(const void* kv_a, mla_dtype kv_dtype, int n_new,
  *   q_nope device [rows, n_heads, 128], q_pe device [rows, n_heads, 64],
  *   w_uk   device [n_heads, 128, 512], q_abs device [rows, n_heads, 576]; all of `dtype`
  *   (F32 or BF16).  rows >= 1, 1 <= n_heads <= 128.
+ *   BF16 runs on the tcgen05 tensor cores (a 128-row GEMM tile per head, fp32
+ *   accumulation, rounded once to bf16); F32 runs on the CUDA cores.
  */
 mla_status mla_absorb_q(const void* q_nope, const void* q_pe, const void* w_uk, void* q_abs,
                         int rows, int n_heads, mla_dtype dtype, cudaStream_t stream);
@@ -178,13 +180,17 @@ mla_status mla_absorb_q(const void* q_nope, const void* q_pe, const void* w_uk, 
  *   lse_part    device float [batch*q_len, n_heads, num_splits]
  *   err_word    device int32 or NULL (MLA_DEVERR_PAGE, MLA_DEVERR_TIMEOUT)
  * Supported: page_size 64; q_dtype F32 with cache F32; q_dtype BF16 with cache
- * BF16 or E4M3.  BF16 runs on the tcgen05 tensor cores (bf16 operands, fp32
- * accumulation, one CTA pair per (query row, split)); F32 runs exact fp32 on
- * the CUDA cores.
+ * BF16 or E4M3.  Both BF16 forms run on the tcgen05 tensor cores (fp32
+ * accumulation, one CTA pair per (query row, split)): a BF16 cache with bf16
+ * operands; an E4M3 cache with f16 operands (the codes widened exactly, the
+ * value rows multiplied by their scale once in f16, q_abs and the softmax
+ * weights rounded to f16), so dequantised values must lie within f16's range.
+ * F32 runs exact fp32 on the CUDA cores.
  * Pool contract: the tensor-core path reads whole 64-row pages.  Rows of a
  * sequence's last page beyond its length, and page 0 (read in place of a
  * block-table entry outside the pool), enter the contraction with zero
- * weight, so they must hold finite values: allocate the pool zero-filled.
+ * weight, so they must hold finite values (no NaN codes for E4M3): allocate
+ * the pool zero-filled.
  */
 mla_status mla_decode_fwd(const void* q_abs, mla_dtype q_dtype, const void* cache,
                           const float* cache_scale, mla_dtype cache_dtype, int num_pages,
@@ -216,6 +222,8 @@ mla_status mla_combine(const float* o_part, const float* lse_part, int rows, int
  *   out[r, h, i] = sum_c W_UV[h, i, c] * o_lat[r, h, c]    (fp32 accumulate)
  *   o_lat device [rows, n_heads, 512], w_uv device [n_heads, 128, 512],
  *   out device [rows, n_heads, 128]; all of `dtype` (F32 or BF16).
+ *   BF16 runs on the tcgen05 tensor cores (a 128-row GEMM tile per head and
+ *   half of the outputs); F32 runs on the CUDA cores.
  */
 mla_status mla_out_uv(const void* o_lat, const void* w_uv, void* out, int rows, int n_heads,
                       mla_dtype dtype, cudaStream_t stream);

@@ -28,6 +28,10 @@ cudaError_t launch_absorb_q(const void* q_nope, const void* q_pe, const void* w_
                             int rows, int n_heads, int dtype, cudaStream_t st);
 cudaError_t launch_out_uv(const void* o_lat, const void* w_uv, void* out, int rows, int n_heads,
                           int dtype, cudaStream_t st);
+// tensor-core versions (bf16): one tcgen05 GEMM per head
+cudaError_t launch_absorb_q_tc(const void* q_nope, const void* q_pe, const void* w_uk, void* q_abs, int rows,
+                               int n_heads, cudaStream_t st);
+cudaError_t launch_out_uv_tc(const void* o_lat, const void* w_uv, void* out, int rows, int n_heads, cudaStream_t st);
 
 struct DecodeArgs {
   const void* q_abs; int q_dtype;

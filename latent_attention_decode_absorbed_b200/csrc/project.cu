@@ -16,6 +16,9 @@ namespace mla {
 namespace {
 
 constexpr int kRB = 8;        // query rows per CTA
+// bf16 projections run on the tensor cores (project_tc.cu); the CUDA-core
+// kernels below serve fp32
+constexpr bool kUseTensorCores = true;
 constexpr int kThr = 128;     // threads per CTA
 
 // 16-byte vector of T, widened to float
@@ -196,6 +199,7 @@ __global__ void __launch_bounds__(kThr) out_uv_kernel(const T* __restrict__ o_la
 cudaError_t launch_absorb_q(const void* q_nope, const void* q_pe, const void* w_uk, void* q_abs,
                             int rows, int n_heads, int dtype, cudaStream_t st) {
   if (rows == 0) return cudaSuccess;
+  if (dtype == MLA_BF16 && kUseTensorCores) return launch_absorb_q_tc(q_nope, q_pe, w_uk, q_abs, rows, n_heads, st);
   dim3 grid(n_heads, (rows + kRB - 1) / kRB, MLA_D_C / 128);
   if (dtype == MLA_F32)
     absorb_q_kernel<float><<<grid, kThr, 0, st>>>((const float*)q_nope, (const float*)q_pe,
@@ -210,6 +214,7 @@ cudaError_t launch_absorb_q(const void* q_nope, const void* q_pe, const void* w_
 cudaError_t launch_out_uv(const void* o_lat, const void* w_uv, void* out, int rows, int n_heads,
                           int dtype, cudaStream_t st) {
   if (rows == 0) return cudaSuccess;
+  if (dtype == MLA_BF16 && kUseTensorCores) return launch_out_uv_tc(o_lat, w_uv, out, rows, n_heads, st);
   dim3 grid(n_heads, (rows + kRB - 1) / kRB, MLA_D_V / 32);
   if (dtype == MLA_F32)
     out_uv_kernel<float><<<grid, kThr, 0, st>>>((const float*)o_lat, (const float*)w_uv, (float*)out,
