@@ -361,12 +361,20 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    # smaller cases of a workload's shape, for profiler captures (not bench lines)
+    ap.add_argument("--batch", type=int, default=None, help="override the workload's batch (profiling)")
+    ap.add_argument("--seq-len", type=int, default=None, help="override the workload's fixed length (profiling)")
+    ap.add_argument("--split-tokens", type=int, default=None, help="override the split length (profiling)")
     args = ap.parse_args()
     assert args.warmup >= 3, "at least 3 warm-up steps"
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     local_rank = int(os.environ.get("LOCAL_RANK", 0))
     w = W.WORKLOADS[args.workload]
+    over = {k: v for k, v in (("batch", args.batch), ("seq_len", args.seq_len),
+                              ("split_tokens", args.split_tokens)) if v is not None}
+    if over:
+        w = W.with_overrides(w, name=w.name + "-profile-case", **over)
     if args.impl == "reference":
         return run_reference(args, w, rank, world)
     if world > 1:

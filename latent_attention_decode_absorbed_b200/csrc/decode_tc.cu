@@ -134,11 +134,13 @@ struct Bars {
   static constexpr int q_full = base + 8;            //       leader: Q of both CTAs loaded
   static constexpr int l_full = base + 9;            //       both: the peer's row sums arrived
   static constexpr int p_free = base + 10;           // [6]   both: O^T MMAs done with a P^T chunk slot
+  static constexpr int q_free = base + 16;           //       both: the unit's score MMAs done (Q reusable)
+  static constexpr int epi_done = base + 17;         //       leader: both CTAs read O^T out (TMEM reusable)
   // e4m3 cache only
-  static constexpr int q_ready = base + 16;          //       leader: both CTAs converted Q to f16
-  static constexpr int sfull8 = base + 17;           // [NS]  local: TMA bytes of a staging slot
-  static constexpr int sempty8 = base + 17 + NS;     // [NS]  local: converters done with the staging slot
-  static constexpr int end = base + 17 + 2 * NS;
+  static constexpr int q_ready = base + 18;          //       leader: both CTAs converted Q to f16
+  static constexpr int sfull8 = base + 19;           // [NS]  local: TMA bytes of a staging slot
+  static constexpr int sempty8 = base + 19 + NS;     // [NS]  local: converters done with the staging slot
+  static constexpr int end = base + 19 + 2 * NS;
 };
 
 // Sum over the 32 lanes of a warp of each of C per-lane values, returned
@@ -246,17 +248,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
   const uint32_t peer = rank ^ 1u;
   const bool leader = rank == 0;
 
-  // ---- unit: (query row r, split s)
-  const int unit = blockIdx.x >> 1;
+  // ---- units: (query row r, split s), persistent: pair `pair` takes units
+  // pair, pair + n_pairs, ...; every role walks the same sequence, so the
+  // barrier phases are counted globally (ring stages, tiles, units)
   const int S = p.num_splits;
-  const int r = unit / S, s = unit % S;
-  const int b = r / p.q_len, t = r % p.q_len;
-  const int L = p.seq_lens[b];
-  const int n_vis = L - p.q_len + t + 1;
-  const int lo = s * p.split_tokens;
-  const int hi = min(lo + p.split_tokens, n_vis);
-  const int n_tok = hi - lo;
-  const int n_tiles = n_tok > 0 ? (n_tok + kTile - 1) / kTile : 0;
+  const int n_units = p.batch * p.q_len * S;
+  const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+  struct UnitInfo { int r, s, b, lo, hi, n_tiles; };
+  auto unit_at = [&](int u) -> UnitInfo {
+    UnitInfo x;
+    x.r = u / S;
+    x.s = u % S;
+    x.b = x.r / p.q_len;
+    const int t = x.r % p.q_len;
+    const int n_vis = p.seq_lens[x.b] - p.q_len + t + 1;
+    x.lo = x.s * p.split_tokens;
+    x.hi = min(x.lo + p.split_tokens, n_vis);
+    const int n_tok = x.hi - x.lo;
+    x.n_tiles = n_tok > 0 ? (n_tok + kTile - 1) / kTile : 0;
+    return x;
+  };
 
   // ---- set-up: barriers, TMEM, cluster sync
   if (threadIdx.x == 0) {
@@ -279,6 +290,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
     mbar_init(bar(B::p_full), 2 * 4 * kSoftGroups);
     mbar_init(bar(B::o_done), 1);
     mbar_init(bar(B::q_full), 1);
+    mbar_init(bar(B::q_free), 1);
+    mbar_init(bar(B::epi_done), 2 * 4 * kSoftGroups);
     mbar_init(bar(B::l_full), kSoftGroups);
     for (int i = 0; i < LY::kPSlots; ++i) mbar_init(bar(B::p_free + i), 1);
     *abort_flag = 0;
@@ -321,15 +334,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
     ++rg.kc;
     return true;
   };
-  if (n_tiles == 0) {
-    // nothing visible in this split: o = 0, lse = -inf (heads split by rank)
-    for (int i = threadIdx.x; i < p.n_heads * MLA_D_C; i += kThreads) {
-      const int h = i / MLA_D_C, d = i % MLA_D_C;
-      if ((h & 1) != (int)rank) continue;
-      p.o_part[(((size_t)r * p.n_heads + h) * S + s) * MLA_D_C + d] = 0.f;
-      if (d == 0) p.lse_part[((size_t)r * p.n_heads + h) * S + s] = -INFINITY;
-    }
-  } else if (F8 && warp == kWarpProd) {
+  if (F8 && warp == kWarpProd) {
     // ============ TMA producer, e4m3 cache (both CTAs) ============
     // The same stages in the same order as the bf16 producer, but each CTA
     // loads raw e4m3 blocks ([64 rows x 64 bytes], one per lane) into its own
@@ -356,10 +361,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
       if (lane == 0) {
         tma_prefetch_desc(&tm_cache);
         tma_prefetch_desc(&tm_q);
-        mbar_arrive_expect_tx(bar(B::q_full), kChunks * LY::kQChunk);
-        for (int c = 0; c < kChunks; ++c)
-          tma_load_3d(s_q + c * LY::kQChunk, &tm_q, 64 * c, (int)rank * HPW, r, bar(B::q_full));
       }
+      uint32_t uc = 0;
+      bool ok = true;
+      for (int u = pair; u < n_units && ok; u += n_pairs) {
+      const UnitInfo U = unit_at(u);
+      if (U.n_tiles == 0) continue;
+      const int r = U.r, b = U.b, lo = U.lo, hi = U.hi, n_tiles = U.n_tiles;
+      if (lane == 0) {
+        // the previous unit's score MMAs must be done with Q
+        if (uc > 0) ok = mbar_wait<false>(bar(B::q_free), (uc - 1) & 1, abort_flag);
+        if (ok) {
+          mbar_arrive_expect_tx(bar(B::q_full), kChunks * LY::kQChunk);
+          for (int c = 0; c < kChunks; ++c)
+            tma_load_3d(s_q + c * LY::kQChunk, &tm_q, 64 * c, (int)rank * HPW, r, bar(B::q_full));
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
       auto load_s8 = [&](int i) -> bool {
         bool vv;
         const int pg = page_of(p, b, lo + kTile * i + 128 * (int)rank + 64 * (lane & 1), &vv);
@@ -386,11 +405,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
         }
         return true;
       };
-      bool ok = load_s8(0);
+      ok = load_s8(0);
       if (ok && n_tiles > 1) ok = load_s8(1);
       for (int i = 0; i < n_tiles && ok; ++i) {
         if (i + 2 < n_tiles) ok = load_s8(i + 2);
         if (ok) ok = load_o8(i);
+      }
+      ++uc;
       }
     }
   } else if (F8 && warp >= kWarpConv0 && warp < kWarpConv0 + kConvWarps) {
@@ -405,7 +426,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
     if constexpr (F8) {
       const int ct = threadIdx.x - 32 * kWarpConv0;
       constexpr int kCT = 32 * kConvWarps;
-      bool ok = __all_sync(0xffffffffu, mbar_wait<false>(bar(B::q_full), 0, abort_flag));
+      uint32_t kc = 0, uc = 0;
+      bool ok = true;
+      for (int u = pair; u < n_units && ok; u += n_pairs) {
+      const UnitInfo U = unit_at(u);
+      if (U.n_tiles == 0) continue;
+      const int b = U.b, lo = U.lo, hi = U.hi, n_tiles = U.n_tiles;
+      ok = __all_sync(0xffffffffu, mbar_wait<false>(bar(B::q_full), uc & 1, abort_flag));
       if (ok) {
         for (int i = ct; i < kChunks * LY::kQChunk / 16; i += kCT) {
           uint4 v = *reinterpret_cast<const uint4*>(smem + LY::kQ + 16 * i);
@@ -422,7 +449,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(mapa(bar(B::q_ready), 0));
       }
-      uint32_t kc = 0;
       auto convert = [&](int nbox, int scale_page) -> bool {
         // scale_page >= 0: value stage of that page (lane l holds rows l, l + 32)
         float s_lo = 1.f, s_hi = 1.f;
@@ -490,6 +516,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
         if (i + 2 < n_tiles) ok = conv_s();
         if (ok) ok = conv_o(i);
       }
+      ++uc;
+      }
     }
   } else if (warp == kWarpProd) {
     // ============ TMA producer (both CTAs), in the order the MMA consumes ============
@@ -504,11 +532,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
       tma_prefetch_desc(&tm_cache);
       tma_prefetch_desc(&tm_cache2);
       tma_prefetch_desc(&tm_q);
-      const uint32_t q_bar = mapa(bar(B::q_full), 0);
-      if (leader) mbar_arrive_expect_tx(bar(B::q_full), 2u * kChunks * LY::kQChunk);
-      for (int c = 0; c < kChunks; ++c)
-        tma_load_3d_pair(s_q + c * LY::kQChunk, &tm_q, 64 * c, (int)rank * HPW, r, q_bar);
     }
+    uint32_t uc = 0;
+    bool ok = true;
+    for (int u = pair; u < n_units && ok; u += n_pairs) {
+    const UnitInfo U = unit_at(u);
+    if (U.n_tiles == 0) continue;
+    const int r = U.r, b = U.b, lo = U.lo, hi = U.hi, n_tiles = U.n_tiles;
+    if (lane == 0) {
+      // the previous unit's score MMAs must be done with Q (both halves)
+      if (uc > 0) ok = mbar_wait<false>(bar(B::q_free), (uc - 1) & 1, abort_flag);
+      if (ok) {
+        const uint32_t q_bar = mapa(bar(B::q_full), 0);
+        if (leader) mbar_arrive_expect_tx(bar(B::q_full), 2u * kChunks * LY::kQChunk);
+        for (int c = 0; c < kChunks; ++c)
+          tma_load_3d_pair(s_q + c * LY::kQChunk, &tm_q, 64 * c, (int)rank * HPW, r, q_bar);
+      }
+    }
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (!ok) break;
     // L2 residency: this CTA's score rows are re-read (by the peer and by
     // itself) for the value operand two tiles later, so they are loaded
     // evict-last; value loads are the rows' last use and go evict-first.
@@ -546,26 +588,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
       }
       return true;
     };
-    bool ok = load_s(0);
+    ok = load_s(0);
     if (ok && n_tiles > 1) ok = load_s(1);
     for (int i = 0; i < n_tiles && ok; ++i) {
       if (i + 2 < n_tiles) ok = load_s(i + 2);
       if (ok) ok = load_o(i);
     }
+    ++uc;
+    }
   } else if (warp == kWarpMma) {
     // ================= MMA issuer (leader CTA) =================
-    // order: S(0), S(1), then per tile i: S(i+2), O(i) -- the score GEMM runs
-    // two tiles ahead so the softmax of tile i overlaps S(i+1), O(i-1), S(i+2)
+    // Per unit: S(0), S(1), then per tile i: S(i+2), O(i) -- the score GEMM
+    // runs two tiles ahead so the softmax of tile i overlaps S(i+1), O(i-1),
+    // S(i+2).  Across units the next unit's S(0), S(1) run while the softmax
+    // warps read the previous unit's O^T out; its first O^T MMA waits for that.
+    // Tiles are numbered globally (gt + i) for the S^T buffers, the P^T ring
+    // and the per-tile barriers.
     if (leader && lane == 0) {
       // e4m3 cache: the operands are f16 (widened codes, Q and P in f16)
       constexpr uint32_t idS = idesc_f16(256, NH, false, false, F8);
       constexpr uint32_t idO = idesc_f16(256, NH, true, false, F8);
-      bool ok = mbar_wait(bar(F8 ? B::q_ready : B::q_full), 0, abort_flag);
+      uint32_t uc = 0, gt = 0;
+      bool ok = true;
+      for (int u = pair; u < n_units && ok; u += n_pairs) {
+      const UnitInfo U = unit_at(u);
+      if (U.n_tiles == 0) continue;
+      const int lo = U.lo, hi = U.hi, n_tiles = U.n_tiles;
+      ok = mbar_wait(bar(F8 ? B::q_ready : B::q_full), uc & 1, abort_flag);
+      if (!ok) break;
       tc_fence_after();
       auto issue_s = [&](int i) -> bool {
-        const int sb = i & 1;
-        if (i >= 2) {
-          if (!mbar_wait(bar(B::s_free + sb), ((i - 2) >> 1) & 1, abort_flag)) return false;
+        const uint32_t gi = gt + i;
+        const int sb = gi & 1;
+        if (gi >= 2) {
+          if (!mbar_wait(bar(B::s_free + sb), ((gi - 2) >> 1) & 1, abort_flag)) return false;
           tc_fence_after();
         }
         const uint32_t d = tmem + (sb ? kColS1 : kColS0);
@@ -585,15 +641,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
           mma_commit_pair(empty, 0x3);
         }
         mma_commit_pair(bar(B::s_full + sb), 0x3);
+        // the unit's last score GEMM: Q may be replaced once it completes
+        if (i == n_tiles - 1) mma_commit_pair(bar(B::q_free), 0x3);
         return true;
       };
       auto issue_o = [&](int j) -> bool {
-        if (!mbar_wait(bar(B::p_full), j & 1, abort_flag)) return false;
+        const uint32_t gj = gt + j;
+        if (!mbar_wait(bar(B::p_full), gj & 1, abort_flag)) return false;
+        // the accumulator is overwritten by this unit's first O^T MMA: the
+        // previous unit's epilogue must have read it out
+        if (j == 0 && uc > 0 && !mbar_wait(bar(B::epi_done), (uc - 1) & 1, abort_flag)) return false;
         tc_fence_after();
         for (int pg_i = 0; pg_i < 4; ++pg_i) {
-          // P^T chunk pg_i of tile j lives in slot (4j + pg_i) mod kPSlots; its
-          // release is committed even for pages past the end of the split
-          const int pslot = (4 * j + pg_i) % LY::kPSlots;
+          // P^T chunk pg_i of global tile gj lives in slot (4 gj + pg_i) mod
+          // kPSlots; its release is committed even for pages past the end
+          const int pslot = (4 * gj + pg_i) % LY::kPSlots;
           if (lo + kTile * j + 64 * pg_i < hi) {
             uint32_t a0, empty;
             if (!ready(ring, a0, empty)) return false;
@@ -612,11 +674,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
         mma_commit_pair(bar(B::o_done), 0x3);
         return true;
       };
-      if (ok) ok = issue_s(0);
+      ok = issue_s(0);
       if (ok && n_tiles > 1) ok = issue_s(1);
       for (int i = 0; i < n_tiles && ok; ++i) {
         if (i + 2 < n_tiles) ok = issue_s(i + 2);
         if (ok) ok = issue_o(i);
+      }
+      gt += n_tiles;
+      ++uc;
       }
     }
   } else {
@@ -642,18 +707,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
     float* red_g = red + g * 4 * HPG;
     float* alpha = own_max;                    // reused after the tile max is consumed
     volatile int* changed_flag = reinterpret_cast<volatile int*>(misc + LY::kChanged) + g;
-    // running row sums of this warp's 32 rows: chunk k, head C*k + lane % C
-    float l_acc[HPG / C];
-#pragma unroll
-    for (int k = 0; k < HPG / C; ++k) l_acc[k] = 0.f;
     const int kt = 128 * (int)rank + tok;      // row within the pair tile
     const int ke = kt & ~1;
     const int wcol = ke & 63;
     const int pchunk = ke >> 6;                // P^T chunk (64 rows of the tile) this warp writes
+    const int st_id = threadIdx.x - 32 * kWarpSoft0;   // 0 .. 511
+    uint32_t uc = 0, gt = 0;                   // units with tiles done, global tile count
     bool ok = true;
+    for (int u = pair; u < n_units && ok; u += n_pairs) {
+    const UnitInfo U = unit_at(u);
+    const int r = U.r, s = U.s, b = U.b, lo = U.lo, hi = U.hi, n_tiles = U.n_tiles;
+    if (n_tiles == 0) {
+      // nothing visible in this split: o = 0, lse = -inf (heads split by rank)
+      for (int idx = st_id; idx < p.n_heads * MLA_D_C; idx += 32 * 4 * kSoftGroups) {
+        const int h = idx / MLA_D_C, d = idx % MLA_D_C;
+        if ((h & 1) != (int)rank) continue;
+        p.o_part[(((size_t)r * p.n_heads + h) * S + s) * MLA_D_C + d] = 0.f;
+        if (d == 0) p.lse_part[((size_t)r * p.n_heads + h) * S + s] = -INFINITY;
+      }
+      continue;
+    }
+    // running row sums of this warp's 32 rows: chunk k, head C*k + lane % C
+    float l_acc[HPG / C];
+#pragma unroll
+    for (int k = 0; k < HPG / C; ++k) l_acc[k] = 0.f;
     for (int i = 0; i < n_tiles; ++i) {
-      const int sb = i & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait<false>(bar(B::s_full + sb), (i >> 1) & 1, abort_flag));
+      const uint32_t gi = gt + i;              // global tile number: buffers and phases
+      const int sb = gi & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait<false>(bar(B::s_full + sb), (gi >> 1) & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
       const int row = lo + kTile * i + kt;
@@ -692,9 +773,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
         }
       }
       named_barrier(1 + g, 128);
-      const int xb = i & 1;
-      const float* m_prev = m_used + ((i + 1) & 1) * NH + g * HPG;
-      float* m_next = m_used + (i & 1) * NH + g * HPG;
+      const int xb = gi & 1;
+      const float* m_prev = m_used + ((gi + 1) & 1) * NH + g * HPG;   // unused on a unit's first tile
+      float* m_next = m_used + (gi & 1) * NH + g * HPG;
       if (q == 0) {
         for (int h = lane; h < HPG; h += 32) {
           const float tm = fmaxf(fmaxf(red_g[h], red_g[HPG + h]), fmaxf(red_g[2 * HPG + h], red_g[3 * HPG + h]));
@@ -703,11 +784,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
         }
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(mapa(bar(B::mx_full + xb), peer));
-        if (__all_sync(0xffffffffu, mbar_wait(bar(B::mx_full + xb), (i >> 1) & 1, abort_flag))) {
+        if (__all_sync(0xffffffffu, mbar_wait(bar(B::mx_full + xb), (gi >> 1) & 1, abort_flag))) {
           int ch = 0;
           for (int h = lane; h < HPG; h += 32) {
             const float mt = fmaxf(own_max[g * HPG + h], x_max[xb * NH + g * HPG + h]);
-            const float mo = m_prev[h];
+            const float mo = i == 0 ? -INFINITY : m_prev[h];
             const float mn = (mt > mo + kRescaleLog2) ? mt : mo;
             m_next[h] = mn;
             // rescale factor for sums and accumulator kept so far (0 when nothing was kept)
@@ -733,7 +814,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
       // behind from one that is done, so skipping phases here would let the
       // rescale and the epilogue read the accumulator before the last O^T
       // MMAs complete
-      const int pn = 4 * i + pchunk;
+      const int pn = 4 * gi + pchunk;
       const int pslot = pn % LY::kPSlots;
       if (pn >= LY::kPSlots) {
         ok = __all_sync(0xffffffffu,
@@ -742,7 +823,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
       }
       const uint32_t row_base = pslot * LY::kPChunk + (wcol & 7) * 2;
       if (i >= 1) {
-        ok = __all_sync(0xffffffffu, mbar_wait<false>(bar(B::o_done), (i - 1) & 1, abort_flag));
+        ok = __all_sync(0xffffffffu, mbar_wait<false>(bar(B::o_done), (gi - 1) & 1, abort_flag));
         if (!ok) break;
         tc_fence_after();
       }
@@ -796,7 +877,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
       if (lane == 0) mbar_arrive_cluster(mapa(bar(B::p_full), 0));
     }
     // ---- epilogue: normalise O^T by the row sums, write o_part and lse
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait<false>(bar(B::o_done), (n_tiles - 1) & 1, abort_flag));
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait<false>(bar(B::o_done), (gt + n_tiles - 1) & 1, abort_flag));
     if (ok) {
       tc_fence_after();
 #pragma unroll
@@ -812,8 +893,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
         }
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(mapa(bar(B::l_full), peer));
-        if (__all_sync(0xffffffffu, mbar_wait(bar(B::l_full), 0, abort_flag))) {
-          const float* m_fin = m_used + ((n_tiles - 1) & 1) * NH + g * HPG;
+        if (__all_sync(0xffffffffu, mbar_wait(bar(B::l_full), uc & 1, abort_flag))) {
+          const float* m_fin = m_used + ((gt + n_tiles - 1) & 1) * NH + g * HPG;
           for (int h = lane; h < HPG; h += 32) {
             const int hg = g * HPG + h;
             const float lt = l_own[hg] + l_x[hg];
@@ -845,6 +926,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
           }
         }
       }
+      // this warp's part of O^T has been read: the next unit may overwrite it
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa(bar(B::epi_done), 0));
+    }
+    gt += n_tiles;
+    ++uc;
     }
   }
 
@@ -884,6 +972,15 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// CTA pairs that fit on the current device at one pair per two SMs
+long long sm_pairs() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 2)
+    return 1;
+  return sms / 2;
+}
+
 template <int NH, bool F8>
 cudaError_t launch_nh(const DecodeArgs& a, const CUtensorMap& tc, const CUtensorMap& tc2, const CUtensorMap& tq,
                       cudaStream_t st) {
@@ -892,8 +989,18 @@ cudaError_t launch_nh(const DecodeArgs& a, const CUtensorMap& tc, const CUtensor
   if (e != cudaSuccess) return e;
   TcParams p{a.n_heads, a.q_len, a.batch, a.block_table, a.max_pages, a.num_pages, a.seq_lens, a.num_splits,
              a.split_tokens, a.softmax_scale * 1.4426950408889634f, a.cache_scale, a.o_part, a.lse_part, a.err};
+  // Persistent pairs (one per SM pair, each walking units pair, pair + P, ...)
+  // amortise set-up, Q loads, pipeline fill and the epilogue across units,
+  // but assign units statically.  Use them when each pair gets many units and
+  // the last round is nearly full; otherwise (few units per SM pair, where
+  // splits of unequal length would leave pairs idle) launch one pair per unit
+  // and let the hardware scheduler balance.
   const long long units = (long long)a.batch * a.q_len * a.num_splits;
-  dim3 grid((unsigned)(2 * units));
+  const long long P = sm_pairs();
+  const long long rounds = (units + P - 1) / P;
+  const bool persistent = rounds >= 6 && rounds * P * 10 <= units * 11;
+  const long long pairs = persistent ? P : units;
+  dim3 grid((unsigned)(2 * pairs));
   decode_tc_kernel<NH, F8><<<grid, kThreadsT<F8>, LY::kSmem, st>>>(tc, tc2, tq, p);
   return cudaGetLastError();
 }
