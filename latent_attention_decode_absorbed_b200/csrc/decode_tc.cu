@@ -42,6 +42,8 @@
 // softmax of one tile overlaps the tensor work of the next ones.
 #include <math.h>
 
+#include <atomic>
+
 #include "mla_device.cuh"
 #include "mla_internal.h"
 #include "sm100.cuh"
@@ -70,6 +72,7 @@ constexpr float kRescaleLog2 = 8.0f;      // lazy rescale threshold (log2 units)
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
 constexpr int kWarpProd = 0, kWarpMma = 1;
+constexpr int kQN = 8;                         // unit queue depth
 template <bool F8>
 constexpr int kWarpSoft0T = F8 ? 4 : 2;
 
@@ -81,6 +84,8 @@ struct TcParams {
   int num_splits, split_tokens;
   float scale_log2;            // softmax_scale * log2(e)
   const float* cache_scale;    // e4m3 cache: per-row dequantisation scale [num_pages * 64]
+  unsigned* claim;             // unit counter of this launch (0 at launch; reset by the last pair)
+  unsigned* done;              // pairs finished
   float* o_part;
   float* lse_part;
   int32_t* err;
@@ -104,7 +109,8 @@ struct Layout {
   static constexpr int kXMax = kOwnMax + NH * 4;            // float [2][NH]   written by the peer
   static constexpr int kLOwn = kXMax + 2 * NH * 4;          // float [NH]
   static constexpr int kLX = kLOwn + NH * 4;                // float [NH]      written by the peer
-  static constexpr int kMiscBytes = kLX + NH * 4;
+  static constexpr int kUnitQ = kLX + NH * 4;              // int [kQN]: units claimed for the pair
+  static constexpr int kMiscBytes = kUnitQ + 4 * 8;
   // ring of operand stages: as many as fit next to Q, P^T and the misc area (at most 6)
   static constexpr int kFixed = kChunks * kQChunk + kPSlots * kPChunk + kMiscBytes + 1024;
   // (e4m3 cache: each stage also has a staging slot for the raw codes)
@@ -140,7 +146,9 @@ struct Bars {
   static constexpr int q_ready = base + 18;          //       leader: both CTAs converted Q to f16
   static constexpr int sfull8 = base + 19;           // [NS]  local: TMA bytes of a staging slot
   static constexpr int sempty8 = base + 19 + NS;     // [NS]  local: converters done with the staging slot
-  static constexpr int end = base + 19 + 2 * NS;
+  static constexpr int uq_full = base + 19 + 2 * NS;   // [8]   both: unit queue slot written
+  static constexpr int uq_empty = base + 27 + 2 * NS;  // [8]   leader: every consumer read the slot
+  static constexpr int end = base + 35 + 2 * NS;
 };
 
 // Sum over the 32 lanes of a warp of each of C per-lane values, returned
@@ -225,6 +233,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
   constexpr int HPW = LY::HPW;
   constexpr int kThreads = kThreadsT<F8>;
   constexpr int kWarpSoft0 = kWarpSoft0T<F8>;
+  // readers of each unit-queue entry: the peer's producer, the MMA issuer,
+  // the converters and the softmax warps of both CTAs
+  constexpr int kQConsumers = 2 + 2 * 4 * kSoftGroups + (F8 ? 2 * kConvWarps : 0);
   using B = Bars<LY::kSlots>;
   static_assert(B::end <= 64, "barrier area");
 
@@ -248,8 +259,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
   const uint32_t peer = rank ^ 1u;
   const bool leader = rank == 0;
 
-  // ---- units: (query row r, split s), persistent: pair `pair` takes units
-  // pair, pair + n_pairs, ...; every role walks the same sequence, so the
+  // ---- units: (query row r, split s); a persistent pair claims units one at a
+  // time (see claim/next_unit); every role walks the pair's same sequence, so
   // barrier phases are counted globally (ring stages, tiles, units)
   const int S = p.num_splits;
   const int n_units = p.batch * p.q_len * S;
@@ -294,6 +305,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
     mbar_init(bar(B::epi_done), 2 * 4 * kSoftGroups);
     mbar_init(bar(B::l_full), kSoftGroups);
     for (int i = 0; i < LY::kPSlots; ++i) mbar_init(bar(B::p_free + i), 1);
+    for (int i = 0; i < kQN; ++i) {
+      mbar_init(bar(B::uq_full + i), 1);
+      mbar_init(bar(B::uq_empty + i), kQConsumers);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -305,6 +320,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(misc + LY::kTmemSlot);
 
   Ring ring{s_base + LY::kRing, bar(B::full), bar(B::empty), LY::kSlots};
+
+  // ---- the pair's unit sequence: the leader's producer claims units from the
+  // launch's counter (dynamic balance) and posts them, in order, to a queue in
+  // both CTAs; every role reads every entry (-1: no units left)
+  int* unit_q = reinterpret_cast<int*>(misc + LY::kUnitQ);
+  auto claim = [&](uint32_t k) -> int {      // leader producer, lane 0
+    const uint32_t slot = k % kQN;
+    if (k >= kQN && !mbar_wait(bar(B::uq_empty + slot), ((k / kQN) - 1) & 1, abort_flag)) return -2;
+    const unsigned cu = atomicAdd(p.claim, 1u);
+    const int uu = cu < (unsigned)n_units ? (int)cu : -1;
+    *reinterpret_cast<volatile int*>(unit_q + slot) = uu;
+    st_cluster_b32(mapa(smem_u32(unit_q + slot), peer), (uint32_t)uu);
+    mbar_arrive_cluster(bar(B::uq_full + slot));
+    mbar_arrive_cluster(mapa(bar(B::uq_full + slot), peer));
+    return uu;
+  };
+  auto next_unit = [&](uint32_t k, bool whole_warp) -> int {
+    const uint32_t slot = k % kQN;
+    if (!mbar_wait(bar(B::uq_full + slot), (k / kQN) & 1, abort_flag)) return -2;
+    const int uu = *reinterpret_cast<volatile int*>(unit_q + slot);
+    if (whole_warp) __syncwarp();
+    if (lane == 0) mbar_arrive_cluster(mapa(bar(B::uq_empty + slot), 0));
+    return uu;
+  };
+  auto producer_unit = [&](uint32_t k) -> int {   // whole producer warp
+    if (leader) {
+      int uu = 0;
+      if (lane == 0) uu = claim(k);
+      return __shfl_sync(0xffffffffu, uu, 0);
+    }
+    return next_unit(k, true);
+  };
 
   // producer side (whole warp): lane 0 waits for a free slot and posts the
   // expected bytes (leader); the lanes then issue the slot's boxes
@@ -364,7 +411,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
       }
       uint32_t uc = 0;
       bool ok = true;
-      for (int u = pair; u < n_units && ok; u += n_pairs) {
+      for (uint32_t k = 0; ok; ++k) {
+      const int u = producer_unit(k);
+      if (u == -2) { ok = false; break; }
+      if (u < 0) break;
       const UnitInfo U = unit_at(u);
       if (U.n_tiles == 0) continue;
       const int r = U.r, b = U.b, lo = U.lo, hi = U.hi, n_tiles = U.n_tiles;
@@ -428,7 +478,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
       constexpr int kCT = 32 * kConvWarps;
       uint32_t kc = 0, uc = 0;
       bool ok = true;
-      for (int u = pair; u < n_units && ok; u += n_pairs) {
+      for (uint32_t k = 0; ok; ++k) {
+      const int u = next_unit(k, true);
+      if (u == -2) { ok = false; break; }
+      if (u < 0) break;
       const UnitInfo U = unit_at(u);
       if (U.n_tiles == 0) continue;
       const int b = U.b, lo = U.lo, hi = U.hi, n_tiles = U.n_tiles;
@@ -535,7 +588,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
     }
     uint32_t uc = 0;
     bool ok = true;
-    for (int u = pair; u < n_units && ok; u += n_pairs) {
+    for (uint32_t k = 0; ok; ++k) {
+    const int u = producer_unit(k);
+    if (u == -2) { ok = false; break; }
+    if (u < 0) break;
     const UnitInfo U = unit_at(u);
     if (U.n_tiles == 0) continue;
     const int r = U.r, b = U.b, lo = U.lo, hi = U.hi, n_tiles = U.n_tiles;
@@ -610,7 +666,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
       constexpr uint32_t idO = idesc_f16(256, NH, true, false, F8);
       uint32_t uc = 0, gt = 0;
       bool ok = true;
-      for (int u = pair; u < n_units && ok; u += n_pairs) {
+      for (uint32_t k = 0; ok; ++k) {
+      const int u = next_unit(k, false);
+      if (u == -2) { ok = false; break; }
+      if (u < 0) break;
       const UnitInfo U = unit_at(u);
       if (U.n_tiles == 0) continue;
       const int lo = U.lo, hi = U.hi, n_tiles = U.n_tiles;
@@ -714,7 +773,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
     const int st_id = threadIdx.x - 32 * kWarpSoft0;   // 0 .. 511
     uint32_t uc = 0, gt = 0;                   // units with tiles done, global tile count
     bool ok = true;
-    for (int u = pair; u < n_units && ok; u += n_pairs) {
+    for (uint32_t k = 0; ok; ++k) {
+    const int u = next_unit(k, true);
+    if (u == -2) { ok = false; break; }
+    if (u < 0) break;
     const UnitInfo U = unit_at(u);
     const int r = U.r, s = U.s, b = U.b, lo = U.lo, hi = U.hi, n_tiles = U.n_tiles;
     if (n_tiles == 0) {
@@ -926,7 +988,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
           }
         }
       }
-      // this warp's part of O^T has been read: the next unit may overwrite it
+      // this warp's part of O^T has been read: the pair's next unit may overwrite it
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(mapa(bar(B::epi_done), 0));
@@ -942,6 +1004,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
     // let copies and MMAs already in flight land before the memory is released
     const uint64_t t0 = globaltimer();
     while (globaltimer() - t0 < 2000000ull) {
+    }
+  }
+  // the last pair to finish resets the launch's unit counter for the next launch
+  if (leader && threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(p.done, 1u) == (unsigned)(n_pairs - 1)) {
+      atomicExch(p.claim, 0u);
+      atomicExch(p.done, 0u);
     }
   }
   tc_fence_before();
@@ -972,6 +1042,28 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// Unit counters of the persistent decode: one (claim, done) pair per launch in
+// flight, taken round robin from kCounterSlots per device.  A launch starts
+// with both at 0 and its last pair sets them back to 0, so consecutive
+// launches on a stream reuse a slot without a reset.  Launches that run
+// concurrently (different streams) take different slots; more than
+// kCounterSlots decode launches in flight at once on one device would share one.
+constexpr int kCounterSlots = 64;
+__device__ unsigned g_unit_claim[kCounterSlots];
+__device__ unsigned g_unit_done[kCounterSlots];
+
+bool claim_slot(unsigned** claim, unsigned** done) {
+  static std::atomic<unsigned> next{0};
+  void* c = nullptr;
+  void* d = nullptr;
+  if (cudaGetSymbolAddress(&c, g_unit_claim) != cudaSuccess || cudaGetSymbolAddress(&d, g_unit_done) != cudaSuccess)
+    return false;
+  const unsigned i = next.fetch_add(1u) % kCounterSlots;
+  *claim = static_cast<unsigned*>(c) + i;
+  *done = static_cast<unsigned*>(d) + i;
+  return true;
+}
+
 // CTA pairs that fit on the current device at one pair per two SMs
 long long sm_pairs() {
   int dev = 0, sms = 0;
@@ -988,18 +1080,15 @@ cudaError_t launch_nh(const DecodeArgs& a, const CUtensorMap& tc, const CUtensor
   cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<NH, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, LY::kSmem);
   if (e != cudaSuccess) return e;
   TcParams p{a.n_heads, a.q_len, a.batch, a.block_table, a.max_pages, a.num_pages, a.seq_lens, a.num_splits,
-             a.split_tokens, a.softmax_scale * 1.4426950408889634f, a.cache_scale, a.o_part, a.lse_part, a.err};
-  // Persistent pairs (one per SM pair, each walking units pair, pair + P, ...)
-  // amortise set-up, Q loads, pipeline fill and the epilogue across units,
-  // but assign units statically.  Use them when each pair gets many units and
-  // the last round is nearly full; otherwise (few units per SM pair, where
-  // splits of unequal length would leave pairs idle) launch one pair per unit
-  // and let the hardware scheduler balance.
+             a.split_tokens, a.softmax_scale * 1.4426950408889634f, a.cache_scale, nullptr, nullptr,
+             a.o_part, a.lse_part, a.err};
+  // Persistent pairs, one per SM pair, claiming units from a counter of this
+  // launch: set-up, Q loads, pipeline fill and the epilogue are amortised and
+  // overlapped across units, and splits of unequal length still balance.
   const long long units = (long long)a.batch * a.q_len * a.num_splits;
   const long long P = sm_pairs();
-  const long long rounds = (units + P - 1) / P;
-  const bool persistent = rounds >= 6 && rounds * P * 10 <= units * 11;
-  const long long pairs = persistent ? P : units;
+  const long long pairs = units < P ? units : P;
+  if (!claim_slot(&p.claim, &p.done)) return cudaErrorInvalidSymbol;
   dim3 grid((unsigned)(2 * pairs));
   decode_tc_kernel<NH, F8><<<grid, kThreadsT<F8>, LY::kSmem, st>>>(tc, tc2, tq, p);
   return cudaGetLastError();
