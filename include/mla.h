@@ -108,6 +108,15 @@ int mla_version(void);
 mla_status mla_rope_table(double theta, int max_pos, float* cos_out, float* sin_out);
 
 /*
+ * mla_decode_workspace_bytes (host function, no GPU needed)
+ * Bytes of caller workspace mla_decode_fwd needs for its split partials:
+ * o_part (fp32 [batch*q_len, n_heads, num_splits, 512]) plus lse_part (fp32
+ * [batch*q_len, n_heads, num_splits]), i.e. batch*q_len*n_heads*num_splits*513*4.
+ * Returns 0 for non-positive arguments.
+ */
+size_t mla_decode_workspace_bytes(int batch, int q_len, int n_heads, int num_splits);
+
+/*
  * mla_cache_append
  * Writes the cache rows of new tokens ("KV Compression - DeepSeek-V3", "How it
  * works" and "Official code": split the 576-wide wkv_a output [512, 64],

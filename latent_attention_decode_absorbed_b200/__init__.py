@@ -26,6 +26,7 @@ _SIGS = {
     "mla_last_error_message": ("s", ""),
     "mla_version": ("i", ""),
     "mla_rope_table": ("i", "dipp"),
+    "mla_decode_workspace_bytes": ("z", "iiii"),
     "mla_cache_append": ("i", "piipppiiipfppippiipp"),
     "mla_absorb_q": ("i", "ppppiiip"),
     "mla_decode_fwd": ("i", "pippiipiipiiiiifpppp"),
@@ -34,7 +35,7 @@ _SIGS = {
     "mla_decode_static": ("i", "pippiipiipiiiiifpippp"),
 }
 _CT = {"p": ctypes.c_void_p, "i": ctypes.c_int, "f": ctypes.c_float, "d": ctypes.c_double,
-       "s": ctypes.c_char_p}
+       "s": ctypes.c_char_p, "z": ctypes.c_size_t}
 
 _lib = None
 
@@ -109,6 +110,11 @@ def unpack_cache_rows(cache):
 
 def mla_version() -> int:
     return lib().mla_version()
+
+
+def mla_decode_workspace_bytes(batch: int, q_len: int, n_heads: int, num_splits: int) -> int:
+    """Bytes of the fp32 split partials (o_part + lse_part) mla_decode_fwd writes."""
+    return int(lib().mla_decode_workspace_bytes(int(batch), int(q_len), int(n_heads), int(num_splits)))
 
 
 def mla_rope_table(theta: float, max_pos: int, cos_out, sin_out):

@@ -1,5 +1,5 @@
-// Split-KV latent attention on the tcgen05 tensor cores (bf16 operands,
-// fp32 accumulation), one CTA pair per (query row, split).
+// Split-KV latent attention on the tcgen05 tensor cores (fp32 accumulation):
+// CTA pairs, each working through (query row, split) units.
 //
 // What it computes ("DeepSeek-V2: MLA Explained", "MLA Full Formulas" part 3
 // with the absorption of "Optimization Note"): for each head h of query row
@@ -27,19 +27,25 @@
 // columns] K-major per chunk, one box per page, issued by four lanes) or one
 // page of the value operand (two 16 KB boxes: [64 rows x this CTA's 128 dims]
 // read MN-major, one per dims block); the value loads of the peer's rows hit
-// L2.  The pool is page-blocked, so every box is a contiguous read.
+// L2 (score loads are evict-last, value loads evict-first).  The pool is
+// page-blocked, so every box is a contiguous read.  With an e4m3 cache the
+// producer loads raw codes into a staging ring and converter warps widen them
+// to f16 (value rows times their scale) into the same operand layout.
 // Warp roles per CTA: 0 TMA producer and TMEM allocator, 1 MMA issuer
-// (leader CTA only), 2-9 softmax (two warpgroups, one per half of the heads;
-// thread = cached row).
+// (leader CTA only), [e4m3: 2-5 converters], then 16 softmax warps in four
+// warpgroups, a quarter of the heads each (thread = cached row).
 //
 // Softmax per tile: each warp takes the per-head max of its 32 rows with a
 // shuffle butterfly, the 4 warps of a warpgroup combine through shared memory, the
 // pair exchanges its maxima through distributed shared memory, and the
 // running max only moves when the tile max exceeds it by more than 2^8 (the
 // accumulator is rescaled in TMEM then).  P = 2^(u - m) is written as bf16
-// straight into the P^T operand of the CTA that owns those heads.  The MMA
-// issuer keeps the score GEMM two tiles ahead of the value GEMM, so the
-// softmax of one tile overlaps the tensor work of the next ones.
+// (f16 for e4m3) straight into the P^T operand of the CTA that owns those
+// heads, in a ring of 64-row chunks.  The MMA issuer keeps the score GEMM two
+// tiles ahead of the value GEMM, so the softmax of one tile overlaps the
+// tensor work of the next ones.  Pairs are persistent (one per SM pair) and
+// claim units dynamically, so one unit's loads and score GEMMs overlap the
+// previous unit's epilogue.
 #include <math.h>
 
 #include <atomic>
@@ -54,10 +60,10 @@ namespace {
 using namespace sm100;
 
 constexpr int kSoftGroups = 4;           // softmax warpgroups, each a quarter of the heads
-// 18 warps (bf16 cache) or 20 (e4m3 cache: two converter warps): see the role map above
+// 18 warps (bf16 cache) or 22 (e4m3 cache: four converter warps): see the role map above
 template <bool F8>
-constexpr int kThreadsT = 32 * ((F8 ? 4 : 2) + 4 * kSoftGroups);
-constexpr int kWarpConv0 = 2, kConvWarps = 2;  // e4m3 converters
+constexpr int kThreadsT = 32 * ((F8 ? 6 : 2) + 4 * kSoftGroups);
+constexpr int kWarpConv0 = 2, kConvWarps = 4;  // e4m3 converters
 constexpr int kBox8 = 4096;                    // one e4m3 block: 64 rows x 64 bytes
 constexpr int kStage8 = 4 * kBox8;             // e4m3 staging of one stage (at most four blocks)
 constexpr int kSlotBytes = 32768;         // one ring stage
@@ -74,7 +80,7 @@ constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
 constexpr int kWarpProd = 0, kWarpMma = 1;
 constexpr int kQN = 8;                         // unit queue depth
 template <bool F8>
-constexpr int kWarpSoft0T = F8 ? 4 : 2;
+constexpr int kWarpSoft0T = F8 ? 6 : 2;
 
 struct TcParams {
   int n_heads, q_len, batch;

@@ -53,6 +53,11 @@ const char* mla_last_error_message(void) { return g_msg; }
 
 int mla_version(void) { return 10000; }
 
+size_t mla_decode_workspace_bytes(int batch, int q_len, int n_heads, int num_splits) {
+  if (batch <= 0 || q_len <= 0 || n_heads <= 0 || num_splits <= 0) return 0;
+  return (size_t)batch * q_len * n_heads * num_splits * (MLA_D_C + 1) * sizeof(float);
+}
+
 mla_status mla_rope_table(double theta, int max_pos, float* cos_out, float* sin_out) {
   MLA_REQUIRE(cos_out && sin_out, MLA_ERR_INVALID_ARG, "mla_rope_table: null output");
   MLA_REQUIRE(max_pos >= 1, MLA_ERR_INVALID_ARG, "mla_rope_table: max_pos must be >= 1");

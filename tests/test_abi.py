@@ -42,7 +42,8 @@ def _code(param: str) -> str:
 def test_header_declares_the_path():
     names = set(_declarations())
     for n in ["mla_cache_append", "mla_absorb_q", "mla_decode_fwd", "mla_combine", "mla_out_uv",
-              "mla_rope_table", "mla_status_string", "mla_last_error_message", "mla_version"]:
+              "mla_rope_table", "mla_decode_workspace_bytes", "mla_status_string", "mla_last_error_message",
+              "mla_version"]:
         assert n in names
 
 
@@ -132,3 +133,11 @@ def test_other_validation(lib):
     mla.mla_cache_append(None, mla.MLA_BF16, 0, None, None, None, 1, 4, 64, None, 1e-6, None, None, 256,
                          None, None, mla.MLA_BF16, 4, None, 0)
     mla.mla_absorb_q(None, None, None, None, 0, 8, mla.MLA_BF16, 0)
+
+
+def test_decode_workspace_bytes_host(lib):
+    # o_part [B*T, H, S, 512] + lse_part [B*T, H, S], fp32: the long workload's 134 MB + 262 KB
+    assert mla.mla_decode_workspace_bytes(8, 1, 128, 64) == 8 * 128 * 64 * 513 * 4
+    assert mla.mla_decode_workspace_bytes(128, 2, 128, 4) == 256 * 128 * 4 * 513 * 4
+    assert mla.mla_decode_workspace_bytes(0, 1, 128, 4) == 0
+    assert mla.mla_decode_workspace_bytes(1, 1, 16, -1) == 0
