@@ -203,9 +203,14 @@ __device__ __forceinline__ float transpose_max(float* v, int lane) {
   return v[0];
 }
 
-__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
-  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+// Store to the peer CTA's shared memory and signal 4 bytes of completed
+// transaction on the peer's mbarrier (no release fence on the sender side).
+__device__ __forceinline__ void st_async_f32(uint32_t cluster_addr, float v, uint32_t cluster_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(cluster_addr),
+               "r"(__float_as_uint(v)), "r"(cluster_bar)
+               : "memory");
 }
+
 __device__ __forceinline__ void st_cluster_b32(uint32_t addr, uint32_t v) {
   asm volatile("st.shared::cluster.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
@@ -302,7 +307,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(B::s_full + i), 1);
       mbar_init(bar(B::s_free + i), 2 * 4 * kSoftGroups);
-      mbar_init(bar(B::mx_full + i), kSoftGroups);
+      mbar_init(bar(B::mx_full + i), kSoftGroups);   // local expect-tx arrivals + the peer's st.async bytes
     }
     mbar_init(bar(B::p_full), 2 * 4 * kSoftGroups);
     mbar_init(bar(B::o_done), 1);
@@ -845,13 +850,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
       const float* m_prev = m_used + ((gi + 1) & 1) * NH + g * HPG;   // unused on a unit's first tile
       float* m_next = m_used + (gi & 1) * NH + g * HPG;
       if (q == 0) {
+        // exchange tile maxima with the peer's group of the same heads: arm
+        // this CTA's barrier for the peer's HPG values, send ours with st.async
+        // (each store completes its bytes on the peer's barrier)
+        if (lane == 0) mbar_arrive_expect_tx(bar(B::mx_full + xb), HPG * 4);
+        __syncwarp();
+        const uint32_t peer_bar = mapa(bar(B::mx_full + xb), peer);
         for (int h = lane; h < HPG; h += 32) {
           const float tm = fmaxf(fmaxf(red_g[h], red_g[HPG + h]), fmaxf(red_g[2 * HPG + h], red_g[3 * HPG + h]));
           own_max[g * HPG + h] = tm;
-          st_cluster_f32(mapa(smem_u32(x_max + xb * NH + g * HPG + h), peer), tm);
+          st_async_f32(mapa(smem_u32(x_max + xb * NH + g * HPG + h), peer), tm, peer_bar);
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(mapa(bar(B::mx_full + xb), peer));
         if (__all_sync(0xffffffffu, mbar_wait(bar(B::mx_full + xb), (gi >> 1) & 1, abort_flag))) {
           int ch = 0;
           for (int h = lane; h < HPG; h += 32) {
@@ -954,13 +963,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
       named_barrier(1 + g, 128);
       float* inv_l = own_max;
       if (q == 0) {
+        // exchange row sums with the peer's group (as the tile maxima)
+        if (lane == 0) mbar_arrive_expect_tx(bar(B::l_full), HPG * 4);
+        __syncwarp();
+        const uint32_t peer_bar = mapa(bar(B::l_full), peer);
         for (int h = lane; h < HPG; h += 32) {
           const float lt = red_g[h] + red_g[HPG + h] + red_g[2 * HPG + h] + red_g[3 * HPG + h];
           l_own[g * HPG + h] = lt;
-          st_cluster_f32(mapa(smem_u32(l_x + g * HPG + h), peer), lt);
+          st_async_f32(mapa(smem_u32(l_x + g * HPG + h), peer), lt, peer_bar);
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(mapa(bar(B::l_full), peer));
         if (__all_sync(0xffffffffu, mbar_wait(bar(B::l_full), uc & 1, abort_flag))) {
           const float* m_fin = m_used + ((gt + n_tiles - 1) & 1) * NH + g * HPG;
           for (int h = lane; h < HPG; h += 32) {
