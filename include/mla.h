@@ -178,7 +178,10 @@ mla_status mla_absorb_q(const void* q_nope, const void* q_pe, const void* w_uk, 
  *   z_j = softmax_scale * (q_abs[r,h,0:512] . c_j + q_abs[r,h,512:576] . k_j)
  *         (E4M3 cache: c_j, k_j are codes times cache_scale[j])
  *   o_part[r,h,s,:] = sum_j e^{z_j - m} c_j / sum_j e^{z_j - m}   over the split's visible j
- *   lse_part[r,h,s] = m + ln sum_j e^{z_j - m}  (natural log; -inf and o = 0 for an empty split)
+ *   lse_part[r,h,s] = m + ln sum_j e^{z_j - m}  (natural log)
+ *   A split with no visible row gets lse_part = -inf; its o_part is left
+ *   unwritten by the tensor-core path (zero on the fp32 path), and
+ *   mla_combine gives it weight 0 without reading it.
  *   q_abs       device [batch*q_len, n_heads, 576], q_dtype F32 or BF16
  *   cache       device [num_pages, 9, 64, 64], page-blocked; cache_scale as for mla_cache_append
  *   block_table device int32 [batch, max_pages_per_seq]

@@ -791,13 +791,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
     const UnitInfo U = unit_at(u);
     const int r = U.r, s = U.s, b = U.b, lo = U.lo, hi = U.hi, n_tiles = U.n_tiles;
     if (n_tiles == 0) {
-      // nothing visible in this split: o = 0, lse = -inf (heads split by rank)
-      for (int idx = st_id; idx < p.n_heads * MLA_D_C; idx += 32 * 4 * kSoftGroups) {
-        const int h = idx / MLA_D_C, d = idx % MLA_D_C;
-        if ((h & 1) != (int)rank) continue;
-        p.o_part[(((size_t)r * p.n_heads + h) * S + s) * MLA_D_C + d] = 0.f;
-        if (d == 0) p.lse_part[((size_t)r * p.n_heads + h) * S + s] = -INFINITY;
-      }
+      // nothing visible in this split: lse = -inf (the leader CTA), o_part is
+      // left unwritten (the merge gives such a split weight 0 and skips it)
+      if (leader)
+        for (int h = st_id; h < p.n_heads; h += 32 * 4 * kSoftGroups)
+          p.lse_part[((size_t)r * p.n_heads + h) * S + s] = -INFINITY;
       continue;
     }
     // running row sums of this warp's 32 rows: chunk k, head C*k + lane % C
