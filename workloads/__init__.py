@@ -67,7 +67,7 @@ WORKLOADS: Dict[str, Workload] = {
     "v3_b1": Workload("v3_b1", 1, 1, 128, 4096, None, "bf16", "bf16", False, 128),
     "serving": Workload("serving", 64, 1, 128, None, (1024, 8192), "bf16", "bf16", True, 2048),
     "long": Workload("long", 8, 1, 128, 131072, None, "bf16", "bf16", True, 2048),
-    "fp8_mtp": Workload("fp8_mtp", 128, 2, 128, 4096, None, "bf16", "e4m3", True, 1024),
+    "fp8_mtp": Workload("fp8_mtp", 128, 2, 128, 4096, None, "bf16", "e4m3", True, 2048),
 }
 WORKLOAD_ORDER: List[str] = ["tiny", "v3_b1", "serving", "long", "fp8_mtp"]
 
