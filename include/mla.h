@@ -26,6 +26,8 @@
  *   mla_absorb_q      q_nope, q_pe  -> q_abs = [W_UK^T q_nope ; q_pe]   (576 per head)
  *   mla_decode_fwd    q_abs, cache  -> split-KV partials (o_part, lse_part)
  *   mla_combine       partials      -> o_lat (512 per head), lse
+ *   (mla_combine_shards: the same merge over the per-GPU results of sequences
+ *    whose cached rows are sharded across GPUs)
  *   mla_out_uv        o_lat         -> out = W_UV o_lat                 (128 per head)
  *
  * Conventions for every entry point
@@ -225,6 +227,26 @@ mla_status mla_decode_fwd(const void* q_abs, mla_dtype q_dtype, const void* cach
 mla_status mla_combine(const float* o_part, const float* lse_part, int rows, int n_heads,
                        int num_splits, void* o_lat, mla_dtype o_dtype, float* lse_out,
                        cudaStream_t stream);
+
+/*
+ * mla_combine_shards
+ * The same log-sum-exp merge over the per-GPU results of sequences whose
+ * cached rows are sharded across GPUs: shard g attended over its own disjoint
+ * row range and merged its splits with mla_combine (o_dtype F32, lse_out
+ * given), and the shards' results were gathered in shard order, e.g. by an
+ * all-gather along the first dimension:
+ *   M = max_g lse_shard[g,r,h];  w_g = e^{lse_g - M}  (0 for lse_g = -inf)
+ *   o_lat[r,h,:] = sum_g w_g o_shard[g,r,h,:] / sum_g w_g,   lse_out[r,h] = M + ln sum_g w_g
+ *   o_shard   device float [num_shards, rows, n_heads, 512]
+ *   lse_shard device float [num_shards, rows, n_heads]
+ *   o_lat     device [rows, n_heads, 512] of o_dtype (F32 or BF16)
+ *   lse_out   device float [rows, n_heads] or NULL
+ * A shard that saw no row of a query (lse = -inf) gets weight 0 and its o is
+ * not read; a (row, head) no shard saw gives o_lat = 0 and lse_out = -inf.
+ */
+mla_status mla_combine_shards(const float* o_shard, const float* lse_shard, int num_shards, int rows,
+                              int n_heads, void* o_lat, mla_dtype o_dtype, float* lse_out,
+                              cudaStream_t stream);
 
 /*
  * mla_out_uv

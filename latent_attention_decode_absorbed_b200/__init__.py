@@ -31,6 +31,7 @@ _SIGS = {
     "mla_absorb_q": ("i", "ppppiiip"),
     "mla_decode_fwd": ("i", "pippiipiipiiiiifpppp"),
     "mla_combine": ("i", "ppiiipipp"),
+    "mla_combine_shards": ("i", "ppiiipipp"),
     "mla_out_uv": ("i", "pppiiip"),
     "mla_decode_static": ("i", "pippiipiipiiiiifpippp"),
 }
@@ -153,6 +154,13 @@ def mla_combine(o_part, lse_part, rows, n_heads, num_splits, o_lat, o_dtype, lse
     _check("mla_combine", lib().mla_combine(_ptr(o_part), _ptr(lse_part), int(rows), int(n_heads),
                                             int(num_splits), _ptr(o_lat), int(o_dtype), _ptr(lse_out),
                                             _stream(stream)))
+
+
+def mla_combine_shards(o_shard, lse_shard, num_shards, rows, n_heads, o_lat, o_dtype, lse_out=None,
+                       stream=None):
+    _check("mla_combine_shards", lib().mla_combine_shards(_ptr(o_shard), _ptr(lse_shard), int(num_shards),
+                                                          int(rows), int(n_heads), _ptr(o_lat), int(o_dtype),
+                                                          _ptr(lse_out), _stream(stream)))
 
 
 def mla_out_uv(o_lat, w_uv, out, rows, n_heads, dtype, stream=None):

@@ -4,6 +4,9 @@
 // splits exactly over disjoint row ranges: with each split's normalised
 // output o_s and log-normaliser lse_s, the full output is the lse-weighted
 // mean of the o_s.  One CTA per (query row, head); 128 threads x 4 channels.
+// The same merge serves two layouts of the parts: the splits of one decode
+// launch ([rows, heads, splits, 512]) and the per-GPU results of a sequence
+// whose rows are sharded across GPUs ([shards, rows, heads, 512]).
 #include <math.h>
 
 #include "mla_device.cuh"
@@ -12,17 +15,23 @@
 namespace mla {
 namespace {
 
+// Strides (in floats) between the parts of one (row, head) and between
+// consecutive (row, head) pairs, for o (multiples of 4) and for lse.
+struct PartStrides {
+  size_t o_part, o_rh, l_part, l_rh;
+};
+
 template <typename OT>
 __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ o_part,
-                                                      const float* __restrict__ lse_part, int S,
+                                                      const float* __restrict__ lse_part, int S, PartStrides st,
                                                       OT* __restrict__ o_lat, float* __restrict__ lse_out) {
   extern __shared__ float w[];               // [S] weights
   __shared__ float red[4];
   const size_t rh = blockIdx.x;
-  const float* lp = lse_part + rh * S;
+  const float* lp = lse_part + rh * st.l_rh;
   // max over splits
   float mx = -INFINITY;
-  for (int s = threadIdx.x; s < S; s += blockDim.x) mx = fmaxf(mx, lp[s]);
+  for (int s = threadIdx.x; s < S; s += blockDim.x) mx = fmaxf(mx, lp[s * st.l_part]);
   mx = warp_max(mx);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
   __syncthreads();
@@ -30,7 +39,7 @@ __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ 
   __syncthreads();
   float sum = 0.f;
   for (int s = threadIdx.x; s < S; s += blockDim.x) {
-    const float v = lp[s];
+    const float v = lp[s * st.l_part];
     const float ws = (mx == -INFINITY || v == -INFINITY) ? 0.f : expf(v - mx);
     w[s] = ws;
     sum += ws;
@@ -40,12 +49,12 @@ __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ 
   __syncthreads();
   sum = red[0] + red[1] + red[2] + red[3];
   const float inv = sum > 0.f ? 1.0f / sum : 0.f;
-  const float4* op = reinterpret_cast<const float4*>(o_part + rh * (size_t)S * MLA_D_C) + threadIdx.x;
+  const float4* op = reinterpret_cast<const float4*>(o_part + rh * st.o_rh) + threadIdx.x;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int s = 0; s < S; ++s) {
     const float ws = w[s];
     if (ws == 0.f) continue;
-    const float4 v = op[(size_t)s * (MLA_D_C / 4)];
+    const float4 v = op[(size_t)s * (st.o_part / 4)];
     acc.x = fmaf(ws, v.x, acc.x); acc.y = fmaf(ws, v.y, acc.y);
     acc.z = fmaf(ws, v.z, acc.z); acc.w = fmaf(ws, v.w, acc.w);
   }
@@ -58,15 +67,18 @@ __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ 
 }  // namespace
 
 cudaError_t launch_combine(const float* o_part, const float* lse_part, int rows, int n_heads,
-                           int num_splits, void* o_lat, int o_dtype, float* lse_out,
+                           int num_parts, bool shard_major, void* o_lat, int o_dtype, float* lse_out,
                            cudaStream_t st) {
   const size_t n = (size_t)rows * n_heads;
   if (n == 0) return cudaSuccess;
-  const size_t smem = (size_t)num_splits * sizeof(float);
+  const size_t smem = (size_t)num_parts * sizeof(float);
+  // splits of one launch: [rows, heads, parts, 512]; shards: [parts, rows, heads, 512]
+  const PartStrides ps = shard_major ? PartStrides{n * MLA_D_C, MLA_D_C, n, 1}
+                                     : PartStrides{MLA_D_C, (size_t)num_parts * MLA_D_C, 1, (size_t)num_parts};
   if (o_dtype == MLA_F32)
-    combine_kernel<float><<<(unsigned)n, 128, smem, st>>>(o_part, lse_part, num_splits, (float*)o_lat, lse_out);
+    combine_kernel<float><<<(unsigned)n, 128, smem, st>>>(o_part, lse_part, num_parts, ps, (float*)o_lat, lse_out);
   else
-    combine_kernel<__nv_bfloat16><<<(unsigned)n, 128, smem, st>>>(o_part, lse_part, num_splits,
+    combine_kernel<__nv_bfloat16><<<(unsigned)n, 128, smem, st>>>(o_part, lse_part, num_parts, ps,
                                                                   (__nv_bfloat16*)o_lat, lse_out);
   return cudaGetLastError();
 }

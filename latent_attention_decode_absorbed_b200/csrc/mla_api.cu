@@ -179,8 +179,25 @@ mla_status mla_combine(const float* o_part, const float* lse_part, int rows, int
   MLA_REQUIRE(o_part && lse_part && o_lat, MLA_ERR_INVALID_ARG, "mla_combine: null pointer");
   MLA_REQUIRE(aligned(o_part, 16) && aligned(o_lat, 16), MLA_ERR_INVALID_ARG,
               "mla_combine: o_part and o_lat must be 16-byte aligned");
-  return cuda_status(launch_combine(o_part, lse_part, rows, n_heads, num_splits, o_lat, o_dtype, lse_out, stream),
+  return cuda_status(launch_combine(o_part, lse_part, rows, n_heads, num_splits, false, o_lat, o_dtype, lse_out,
+                                    stream),
                      "mla_combine launch");
+}
+
+mla_status mla_combine_shards(const float* o_shard, const float* lse_shard, int num_shards, int rows,
+                              int n_heads, void* o_lat, mla_dtype o_dtype, float* lse_out, cudaStream_t stream) {
+  MLA_REQUIRE(rows >= 0 && n_heads >= 1 && n_heads <= MLA_MAX_HEADS && num_shards >= 1, MLA_ERR_INVALID_ARG,
+              "mla_combine_shards: need rows >= 0, n_heads in [1, %d], num_shards >= 1", MLA_MAX_HEADS);
+  MLA_REQUIRE(o_dtype == MLA_F32 || o_dtype == MLA_BF16, MLA_ERR_UNSUPPORTED,
+              "mla_combine_shards: o_dtype must be F32 or BF16");
+  MLA_REQUIRE(num_shards <= 8192, MLA_ERR_UNSUPPORTED, "mla_combine_shards: num_shards above 8192");
+  if (rows == 0) return MLA_OK;
+  MLA_REQUIRE(o_shard && lse_shard && o_lat, MLA_ERR_INVALID_ARG, "mla_combine_shards: null pointer");
+  MLA_REQUIRE(aligned(o_shard, 16) && aligned(o_lat, 16), MLA_ERR_INVALID_ARG,
+              "mla_combine_shards: o_shard and o_lat must be 16-byte aligned");
+  return cuda_status(launch_combine(o_shard, lse_shard, rows, n_heads, num_shards, true, o_lat, o_dtype, lse_out,
+                                    stream),
+                     "mla_combine_shards launch");
 }
 
 }  // extern "C"

@@ -46,8 +46,10 @@ cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t st);
 bool decode_tc_supported(const DecodeArgs& a);
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st);
 
+// shard_major: parts laid out [num_parts, rows, n_heads, 512] (per-GPU results
+// of a row-sharded sequence) instead of [rows, n_heads, num_parts, 512]
 cudaError_t launch_combine(const float* o_part, const float* lse_part, int rows, int n_heads,
-                           int num_splits, void* o_lat, int o_dtype, float* lse_out,
+                           int num_parts, bool shard_major, void* o_lat, int o_dtype, float* lse_out,
                            cudaStream_t st);
 
 }  // namespace mla

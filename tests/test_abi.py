@@ -129,6 +129,16 @@ def test_other_validation(lib):
         mla.mla_cache_append(FAKE, mla.MLA_BF16, 8, FAKE, FAKE, FAKE, 1, 4, 64, None, -1.0, FAKE, FAKE, 256,
                              FAKE, None, mla.MLA_BF16, 4, None, 0)
     assert e.value.status == mla.MLA_ERR_INVALID_ARG       # negative eps
+    with pytest.raises(mla.MlaError) as e:
+        mla.mla_combine_shards(FAKE, None, 2, 4, 8, FAKE, mla.MLA_F32, None, 0)
+    assert e.value.status == mla.MLA_ERR_INVALID_ARG       # null lse_shard
+    with pytest.raises(mla.MlaError) as e:
+        mla.mla_combine_shards(FAKE, FAKE, 0, 4, 8, FAKE, mla.MLA_F32, None, 0)
+    assert e.value.status == mla.MLA_ERR_INVALID_ARG       # no shards
+    with pytest.raises(mla.MlaError) as e:
+        mla.mla_combine_shards(FAKE, FAKE, 2, 4, 8, FAKE, mla.MLA_E4M3, None, 0)
+    assert e.value.status == mla.MLA_ERR_UNSUPPORTED
+    mla.mla_combine_shards(None, None, 2, 0, 8, None, mla.MLA_F32, None, 0)   # zero rows
     # zero-size work is accepted and enqueues nothing (no GPU touched)
     mla.mla_cache_append(None, mla.MLA_BF16, 0, None, None, None, 1, 4, 64, None, 1e-6, None, None, 256,
                          None, None, mla.MLA_BF16, 4, None, 0)
