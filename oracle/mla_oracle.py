@@ -22,7 +22,7 @@ blocking, fusion or reordering beyond what their formulas state.  Sources
            max 448, no infinities, NaN = S.1111.111); used for the e4m3 cache
            with one fp32 scale per token (absmax/448).
 
-Readings where the pages are silent (each listed in the design doc):
+Readings where the pages are silent:
   * RoPE pairs channels (2i, 2i+1), angle = pos * theta^(-2i/64), theta=1e4,
     rotation [x0 cos - x1 sin, x0 sin + x1 cos].
   * RMSNorm(x) = x / sqrt(mean(x^2) + eps) * gain, eps = 1e-6.

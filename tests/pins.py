@@ -301,6 +301,32 @@ def pin_cache_rows():
     np.testing.assert_allclose(pn(rows[:, 512:]), pn(kv[:, 512:]), rtol=1e-13)
 
 
+def pin_normwise_rel_err():
+    """The parity gate: max over (t, h) of ||got - ref||_2 / ||ref||_2 over the
+    last axis, checked on hand-computed values.  Head 0 of token 0 has ref
+    (3, 4), norm 5, and error (0, 1): ratio 0.2; head 1 has ref (1, 0) and
+    error (0.5, 0): ratio 0.5; token 1 has ratios 0.25 and 0.6.  The answer
+    is 0.6.  A mean (0.3875), the norm taken over the wrong axis, a
+    denominator taken from `got`, one global norm ratio (0.44) or a constant 0
+    all give something else."""
+    ref = np.array([[[3.0, 4.0], [1.0, 0.0]],
+                    [[0.0, 2.0], [5.0, 0.0]]])
+    got = np.array([[[3.0, 5.0], [1.5, 0.0]],
+                    [[0.0, 2.5], [5.0, 3.0]]])
+    # token 1: head 0 error 0.5 over norm 2 -> 0.25; head 1 error 3 over norm 5 -> 0.6
+    err = oracle.normwise_rel_err(got, ref)
+    assert abs(err - 0.6) < 1e-15, err
+    assert oracle.normwise_rel_err(ref, ref) == 0.0
+    # scale invariance, and the argument order matters (ref is the denominator)
+    assert abs(oracle.normwise_rel_err(7.0 * got, 7.0 * ref) - 0.6) < 1e-15
+    swapped = oracle.normwise_rel_err(ref, got)
+    assert abs(swapped - max(1 / np.hypot(3, 5), 0.5 / 1.5, 0.5 / np.hypot(0, 2.5), 3 / np.hypot(5, 3))) < 1e-15
+    # one (t, h) far off dominates however many are exact
+    big = np.ones((3, 5, 16)); off = big.copy(); off[2, 4, 0] += 16.0
+    assert abs(oracle.normwise_rel_err(off, big) - 4.0) < 1e-15
+
+
 ALL_PINS = [pin_cache_arithmetic, pin_rmsnorm, pin_rope, pin_e4m3, pin_bf16_rounding,
             pin_naive_equals_absorbed, pin_single_row, pin_uniform_scores, pin_two_rows_sigmoid,
-            pin_row_permutation, pin_causal, pin_brute_force, pin_split_combine, pin_cache_rows]
+            pin_row_permutation, pin_causal, pin_brute_force, pin_split_combine, pin_cache_rows,
+            pin_normwise_rel_err]

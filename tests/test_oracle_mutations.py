@@ -12,7 +12,8 @@ import pins
 
 ORIG = {name: getattr(om, name) for name in
         ["attention_naive", "attention_absorbed", "rope_angles", "rope", "rms_norm",
-         "e4m3_encode", "combine_partials", "absorb_q", "out_uv", "round_to_bf16"]}
+         "e4m3_encode", "combine_partials", "absorb_q", "out_uv", "round_to_bf16",
+          "normwise_rel_err"]}
 
 
 def _patch(monkeypatch, name, fn):
@@ -94,9 +95,39 @@ def _bf16_truncates(monkeypatch):
     _patch(monkeypatch, "round_to_bf16", rb)
 
 
+def _gate_mean(monkeypatch):
+    def gate(got, ref):
+        got = np.asarray(got, np.float64); ref = np.asarray(ref, np.float64)
+        return float(np.mean(np.linalg.norm(got - ref, axis=-1) / np.linalg.norm(ref, axis=-1)))
+    _patch(monkeypatch, "normwise_rel_err", gate)
+
+
+def _gate_den_from_got(monkeypatch):
+    _patch(monkeypatch, "normwise_rel_err", lambda got, ref: ORIG["normwise_rel_err"](ref, got))
+
+
+def _gate_wrong_axis(monkeypatch):
+    def gate(got, ref):
+        got = np.asarray(got, np.float64); ref = np.asarray(ref, np.float64)
+        return float(np.max(np.linalg.norm(got - ref, axis=-2) / np.linalg.norm(ref, axis=-2)))
+    _patch(monkeypatch, "normwise_rel_err", gate)
+
+
+def _gate_zero(monkeypatch):
+    _patch(monkeypatch, "normwise_rel_err", lambda got, ref: 0.0)
+
+
+def _gate_global_norm(monkeypatch):
+    def gate(got, ref):
+        got = np.asarray(got, np.float64); ref = np.asarray(ref, np.float64)
+        return float(np.linalg.norm(got - ref) / np.linalg.norm(ref))
+    _patch(monkeypatch, "normwise_rel_err", gate)
+
+
 MUTATIONS = [_drop_rope_term, _scale_128, _rope_wrong_direction, _rope_half_split, _rms_no_sqrt,
              _causal_excludes_self, _e4m3_ties_away, _combine_no_weights, _wrong_value_matrix,
-             _bf16_truncates]
+             _bf16_truncates, _gate_mean, _gate_den_from_got, _gate_wrong_axis, _gate_zero,
+             _gate_global_norm]
 
 
 @pytest.mark.parametrize("mutate", MUTATIONS, ids=lambda f: f.__name__.strip("_"))
