@@ -3,7 +3,10 @@
 // For callers that cannot allocate device memory themselves.  The split
 // partials live in a file-scope device array of fixed size; host code never
 // uses the array's name as a device address but looks the address up once
-// per device with cudaGetSymbolAddress, with that device current.
+// per device (and again if that device's context was replaced, e.g. after
+// cudaDeviceReset) with cudaGetSymbolAddress, with that device current.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "mla.h"
@@ -18,9 +21,42 @@ static __device__ __align__(256) float g_partials[kPartials * MLA_D_C + kPartial
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
-float* g_addr[kMaxDevices] = {};
+// The looked-up address is only valid in the context it was looked up in:
+// after cudaDeviceReset the device gets a new primary context and the array a
+// new address.  Each entry therefore remembers the context's unique id.
+struct ScratchEntry {
+  unsigned long long ctx_id;
+  float* addr;
+};
+ScratchEntry g_addr[kMaxDevices] = {};
 
-// Device address of g_partials on the current device (looked up on first use).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Unique id of the calling thread's current context (0 if it cannot be read).
+unsigned long long current_ctx_id() {
+  static CtxGetCurrentFn get_cur = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<CtxGetCurrentFn>(f);
+    f = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(f);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_cur && get_id && get_cur(&ctx) == CUDA_SUCCESS && ctx && get_id(ctx, &id) == CUDA_SUCCESS) return id;
+  return 0;
+}
+
+// Device address of g_partials on the current device: looked up once per
+// device and context (cudaGetSymbolAddress allocates nothing).
 mla_status scratch_address(float** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
@@ -28,13 +64,16 @@ mla_status scratch_address(float** out) {
   if (dev < 0 || dev >= kMaxDevices)
     return fail(MLA_ERR_UNSUPPORTED, "mla_decode_static: device ordinal %d above %d", dev, kMaxDevices - 1);
   std::lock_guard<std::mutex> lock(g_mu);
-  if (g_addr[dev] == nullptr) {
+  unsigned long long id = current_ctx_id();   // 0 while no context is current yet
+  if (id == 0 || g_addr[dev].addr == nullptr || g_addr[dev].ctx_id != id) {
+    // set-up for this device and context (binds the context if none is current)
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_partials);
     if (e != cudaSuccess) return cuda_status(e, "mla_decode_static: cudaGetSymbolAddress");
-    g_addr[dev] = static_cast<float*>(p);
+    g_addr[dev].addr = static_cast<float*>(p);
+    g_addr[dev].ctx_id = current_ctx_id();
   }
-  *out = g_addr[dev];
+  *out = g_addr[dev].addr;
   return MLA_OK;
 }
 

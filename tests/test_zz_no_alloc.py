@@ -1,6 +1,7 @@
 """mla_decode_static, the entry point for callers that cannot allocate device
 memory themselves (it keeps the split partials in a scratch array the library
-holds), against the workspace path mla_decode_fwd + mla_combine.
+holds), against the workspace path mla_decode_fwd + mla_combine and against
+the fp64 oracle's split partials and combine.
 
 This file is collected last on purpose, so that a run stopping at the first
 failure has already run every other test; it also passes alone in a fresh
@@ -21,7 +22,7 @@ torch = pytest.importorskip("torch")
 TOL = 1e-2          # the bf16-cache parity gate
 
 
-def _problem(seed, lens, T, H, split_tokens):
+def _problem(seed, lens, T, H, split_tokens, host=None):
     g = np.random.default_rng(seed)
     npg = [(L + 63) // 64 for L in lens]
     num_pages = sum(npg) + 1
@@ -30,9 +31,13 @@ def _problem(seed, lens, T, H, split_tokens):
     off = 0
     for b, n in enumerate(npg):
         bt[b, :n] = ids[off:off + n]; off += n
-    cache = to_device(round_bf16(g.standard_normal((num_pages * 64, 576)).astype(np.float32)), "bf16")
-    q = to_device(round_bf16(g.standard_normal((len(lens) * T, H, 576)).astype(np.float32) * 0.25), "bf16")
+    rows = round_bf16(g.standard_normal((num_pages * 64, 576)).astype(np.float32))
+    qh = round_bf16(g.standard_normal((len(lens) * T, H, 576)).astype(np.float32) * 0.25)
+    cache = to_device(rows, "bf16")
+    q = to_device(qh, "bf16")
     S = -(-bt.shape[1] * 64 // split_tokens)
+    if host is not None:
+        host.update(rows=rows, q=qh, bt=bt, lens=list(lens), T=T, S=S, split_tokens=split_tokens)
     return dict(q_abs=q, q_dtype=mla.MLA_BF16, cache=mla.pack_cache_rows(cache), cache_scale=None,
                 cache_dtype=mla.MLA_BF16, num_pages=num_pages, block_table=torch.from_numpy(bt).cuda(),
                 max_pages_per_seq=bt.shape[1], page_size=64,
@@ -63,9 +68,26 @@ def _static(p):
     return to_host_f64(o_lat), to_host_f64(lse)
 
 
-def test_static_scratch_matches_workspace_path_on_consecutive_calls():
-    a = _problem(1, [70, 300, 129], 1, 128, 128)
-    b = _problem(2, [5, 1000], 2, 64, 256)
+def _oracle(h):
+    """fp64 oracle: split partials of every sequence, then their combine."""
+    o_all, l_all = [], []
+    T = h["T"]
+    for b, L in enumerate(h["lens"]):
+        slots = np.concatenate([h["bt"][b, j] * 64 + np.arange(64) for j in range((L + 63) // 64)])[:L]
+        c = h["rows"][slots].astype(np.float64)
+        q = h["q"][b * T:(b + 1) * T].astype(np.float64)
+        o, l = oracle.attention_partials(q[..., :512], q[..., 512:], c[:, :512], c[:, 512:],
+                                         h["split_tokens"], h["S"])
+        oc, lc = oracle.combine_partials(o, l)
+        o_all.append(oc); l_all.append(lc)
+    return np.concatenate(o_all), np.concatenate(l_all)
+
+
+def test_static_scratch_matches_workspace_path_and_oracle_on_consecutive_calls():
+    ha, hb = {}, {}
+    a = _problem(1, [70, 300, 129], 1, 128, 128, ha)
+    b = _problem(2, [5, 1000], 2, 64, 256, hb)
+    refs = {id(a): _oracle(ha), id(b): _oracle(hb)}
     # two calls in a row with different shapes, then the first again: the
     # scratch keeps the previous call's contents, which must not leak through
     for p in (a, b, a):
@@ -74,6 +96,26 @@ def test_static_scratch_matches_workspace_path_on_consecutive_calls():
         assert np.all(np.isfinite(got_o)) and np.all(np.isfinite(got_l))
         assert oracle.normwise_rel_err(got_o, ref_o) < TOL
         np.testing.assert_allclose(got_l, ref_l, atol=1e-3)
+        or_o, or_l = refs[id(p)]
+        assert oracle.normwise_rel_err(got_o, or_o) < TOL
+        np.testing.assert_allclose(got_l, or_l, atol=1e-3)
+
+
+def test_static_scratch_at_exactly_its_capacity():
+    # 1 row x 128 heads x 64 splits = 8192 partial rows: the last partial's
+    # o_part row ends where the lse_part area of the scratch begins
+    h = {}
+    p = _problem(4, [64 * 64], 1, 128, 64, h)
+    assert p["batch"] * p["q_len"] * p["n_heads"] * p["num_splits"] == mla.MLA_STATIC_MAX_PARTIALS
+    ref_o, ref_l = _with_workspace(p)
+    for _ in range(2):
+        got_o, got_l = _static(p)
+        assert np.all(np.isfinite(got_o)) and np.all(np.isfinite(got_l))
+        assert oracle.normwise_rel_err(got_o, ref_o) < TOL
+        np.testing.assert_allclose(got_l, ref_l, atol=1e-3)
+    or_o, or_l = _oracle(h)
+    assert oracle.normwise_rel_err(got_o, or_o) < TOL
+    np.testing.assert_allclose(got_l, or_l, atol=1e-3)
 
 
 def test_static_scratch_rejects_requests_above_its_capacity():
