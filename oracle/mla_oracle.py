@@ -33,7 +33,11 @@ Readings where the pages are silent:
     tokens are appended before attending; query t of a sequence with L cached
     rows (new rows included) sits at position L - T + t.
   * W_UK, W_UV are stored [H, 128, 512]: k^C_h = W_UK[h] c, v^C_h = W_UV[h] c.
-  * The path ends at the per-head 128-d outputs (W_O is not applied).
+  * The attention core ends at the per-head 128-d outputs; the output
+    projection u = W_O [o_1; ...; o_H] (out_projection) and the wkv_a
+    projection that produces the cached rows (kv_a_projection) are the
+    steps on either side of it.  W_O is [d, H*128] with head h's element i
+    at column h*128 + i; W_kv,a is [576, d].
   * e4m3 cache: one fp32 scale per token over all 576 values, scale = a/448
     with a = max |x|; code = RNE-satfinite(x * 448 / a); a = 0 -> all zero.
 """
@@ -193,6 +197,25 @@ def cache_rows(kv_a: np.ndarray, pos: np.ndarray, gain=None, eps: float = 1e-6,
     return np.concatenate([c, kr], axis=1)
 
 
+def kv_a_projection(h: np.ndarray, w_kva: np.ndarray) -> np.ndarray:
+    """The joint down-projection that feeds the cache  [V3-KV] "How it works",
+    Eq. (1) and the widened official map: [c_t^KV ; k~_t^R] = W_kv,a h_t, one
+    576-wide row per token (512 latent channels, then the 64 rope channels
+    before RoPE).  h [n, d], w_kva [576, d] -> fp64 [n, 576]."""
+    h = np.asarray(h, np.float64); w_kva = np.asarray(w_kva, np.float64)
+    if w_kva.shape[0] != D_ROW or w_kva.shape[1] != h.shape[1]:
+        raise ValueError("kv_a_projection: w_kva must be [576, d] for h [n, d]")
+    return h @ w_kva.T
+
+
+def cache_rows_from_hidden(h: np.ndarray, w_kva: np.ndarray, pos: np.ndarray, gain=None, eps: float = 1e-6,
+                           theta: float = 10000.0) -> np.ndarray:
+    """Cache rows straight from the hidden states: the wkv_a projection, then
+    the split / RMSNorm / RoPE of cache_rows  [V3-KV] "How it works" and
+    "Official code" (split(wkv_a(x), [512, 64]), kv_norm)."""
+    return cache_rows(kv_a_projection(h, w_kva), pos, gain, eps, theta)
+
+
 def stored_rows(rows: np.ndarray, cache_dtype: str):
     """What a cache of the given storage dtype holds for fp64 rows.
     Returns (values fp64 [n, 576], codes or None, scale or None)."""
@@ -330,6 +353,18 @@ def out_uv(o_lat, w_uv):
     """out[t, i] = W^UV_i o_lat[t, i]  (value up-projection, [V2-C] §2, moved
     after the softmax sum)."""
     return np.einsum("thc,hvc->thv", np.asarray(o_lat, np.float64), np.asarray(w_uv, np.float64))
+
+
+def out_projection(out, w_o):
+    """u_t = W_O [o_{t,1}; o_{t,2}; ...; o_{t,n_h}]  ([V2-C] §3, "Concatenate
+    all heads and project"): the heads' 128-wide outputs are concatenated in
+    head order (element i of head h at h*128 + i) and multiplied by W_O.
+    out [T, H, 128], w_o [d, H*128] -> fp64 [T, d]."""
+    out = np.asarray(out, np.float64); w_o = np.asarray(w_o, np.float64)
+    T, H, dv = out.shape
+    if w_o.shape[1] != H * dv:
+        raise ValueError("out_projection: w_o must be [d, H*128]")
+    return out.reshape(T, H * dv) @ w_o.T
 
 
 # --------------------------------------------------------------------------

@@ -326,7 +326,76 @@ def pin_normwise_rel_err():
     assert abs(oracle.normwise_rel_err(off, big) - 4.0) < 1e-15
 
 
+def pin_out_projection():
+    """u = W_O [o_1; ...; o_H]: identity W_O gives the heads concatenated in
+    head order; a one-hot row of W_O picks out exactly one (head, element);
+    scalar loops agree; and W_O composed with W_UV per head (the value
+    up-projection combined with the output projection) gives the same u."""
+    g = _rng(71)
+    T, H = 2, 3
+    out = g.standard_normal((T, H, 128))
+    # identity: u[t] = [out[t,0,:], out[t,1,:], out[t,2,:]]
+    u = oracle.out_projection(out, np.eye(H * 128))
+    np.testing.assert_array_equal(u, np.concatenate([out[:, h, :] for h in range(H)], axis=1))
+    # one-hot rows: row j of W_O selects element i of head h at column h*128 + i
+    sel = [(0, 5), (1, 0), (2, 127), (1, 77)]
+    w = np.zeros((len(sel), H * 128))
+    for j, (h, i) in enumerate(sel):
+        w[j, h * 128 + i] = 1.0
+    u = oracle.out_projection(out, w)
+    for j, (h, i) in enumerate(sel):
+        np.testing.assert_array_equal(u[:, j], out[:, h, i])
+    # scalar loops on a small non-square W_O
+    d = 5
+    w = g.standard_normal((d, H * 128))
+    u = oracle.out_projection(out, w)
+    for t in range(T):
+        for j in range(d):
+            ref = 0.0
+            for h in range(H):
+                for i in range(128):
+                    ref += w[j, h * 128 + i] * out[t, h, i]
+            assert abs(u[t, j] - ref) <= 1e-12 * (1 + abs(ref))
+    # folding: sum_h (W_O[:, h] W_UV[h]) o_lat[h] == W_O [W_UV o_lat]
+    q_nope, q_pe, w_uk, w_uv, c, kr = _problem(72, T, H, 40)
+    o, o_lat, _ = oracle.attention_absorbed(q_nope, q_pe, w_uk, w_uv, c, kr)
+    u1 = oracle.out_projection(o, w)
+    u2 = sum(o_lat[:, h, :] @ (w[:, h * 128:(h + 1) * 128] @ w_uv[h]).T for h in range(H))
+    np.testing.assert_allclose(u1, u2, rtol=1e-11, atol=1e-13)
+
+
+def pin_kv_a_projection():
+    """[c; k~R] = W_kv,a h: identity W gives h back; a one-hot row picks one
+    hidden channel; scalar loops agree; and the cache rows built from h go
+    through the same [512, 64] split, RMSNorm and RoPE as cache_rows."""
+    g = _rng(73)
+    n = 3
+    h = g.standard_normal((n, 576))
+    np.testing.assert_array_equal(oracle.kv_a_projection(h, np.eye(576)), h)
+    d = 40
+    h = g.standard_normal((n, d))
+    w = np.zeros((576, d))
+    w[0, 7] = 1.0; w[511, 0] = 1.0; w[512, 39] = 1.0; w[575, 3] = 1.0
+    kv = oracle.kv_a_projection(h, w)
+    np.testing.assert_array_equal(kv[:, 0], h[:, 7]); np.testing.assert_array_equal(kv[:, 511], h[:, 0])
+    np.testing.assert_array_equal(kv[:, 512], h[:, 39]); np.testing.assert_array_equal(kv[:, 575], h[:, 3])
+    w = g.standard_normal((576, d))
+    kv = oracle.kv_a_projection(h, w)
+    for t in range(n):
+        for j in (0, 100, 511, 512, 575):
+            ref = sum(w[j, k] * h[t, k] for k in range(d))
+            assert abs(kv[t, j] - ref) <= 1e-12 * (1 + abs(ref))
+    pos = np.array([0, 5, 4095])
+    np.testing.assert_allclose(oracle.cache_rows_from_hidden(h, w, pos), oracle.cache_rows(kv, pos), rtol=0, atol=0)
+    # the latent half is RMS-normalised, the rope half keeps its pair norms
+    rows = oracle.cache_rows_from_hidden(h, w, pos)
+    np.testing.assert_allclose(np.mean(rows[:, :512] ** 2, axis=1),
+                               1.0 / (1.0 + 1e-6 / np.mean(kv[:, :512] ** 2, axis=1)), rtol=1e-12)
+    pn = lambda v: np.hypot(v[..., 0::2], v[..., 1::2])
+    np.testing.assert_allclose(pn(rows[:, 512:]), pn(kv[:, 512:]), rtol=1e-13)
+
+
 ALL_PINS = [pin_cache_arithmetic, pin_rmsnorm, pin_rope, pin_e4m3, pin_bf16_rounding,
             pin_naive_equals_absorbed, pin_single_row, pin_uniform_scores, pin_two_rows_sigmoid,
             pin_row_permutation, pin_causal, pin_brute_force, pin_split_combine, pin_cache_rows,
-            pin_normwise_rel_err]
+            pin_normwise_rel_err, pin_out_projection, pin_kv_a_projection]

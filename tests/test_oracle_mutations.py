@@ -13,7 +13,7 @@ import pins
 ORIG = {name: getattr(om, name) for name in
         ["attention_naive", "attention_absorbed", "rope_angles", "rope", "rms_norm",
          "e4m3_encode", "combine_partials", "absorb_q", "out_uv", "round_to_bf16",
-          "normwise_rel_err"]}
+          "normwise_rel_err", "out_projection", "kv_a_projection"]}
 
 
 def _patch(monkeypatch, name, fn):
@@ -124,10 +124,25 @@ def _gate_global_norm(monkeypatch):
     _patch(monkeypatch, "normwise_rel_err", gate)
 
 
+def _concat_interleaved(monkeypatch):
+    def proj(out, w_o):
+        out = np.asarray(out, np.float64)
+        T, H, dv = out.shape
+        return out.transpose(0, 2, 1).reshape(T, H * dv) @ np.asarray(w_o, np.float64).T   # i*H + h order
+    _patch(monkeypatch, "out_projection", proj)
+
+
+def _kv_a_transposed_halves(monkeypatch):
+    def proj(h, w):
+        kv = ORIG["kv_a_projection"](h, w)
+        return np.concatenate([kv[:, 64:], kv[:, :64]], axis=1)      # rope channels first
+    _patch(monkeypatch, "kv_a_projection", proj)
+
+
 MUTATIONS = [_drop_rope_term, _scale_128, _rope_wrong_direction, _rope_half_split, _rms_no_sqrt,
              _causal_excludes_self, _e4m3_ties_away, _combine_no_weights, _wrong_value_matrix,
              _bf16_truncates, _gate_mean, _gate_den_from_got, _gate_wrong_axis, _gate_zero,
-             _gate_global_norm]
+             _gate_global_norm, _concat_interleaved, _kv_a_transposed_halves]
 
 
 @pytest.mark.parametrize("mutate", MUTATIONS, ids=lambda f: f.__name__.strip("_"))
