@@ -198,8 +198,17 @@ mla_status mla_absorb_q(const void* q_nope, const void* q_pe, const void* w_uk, 
  * accumulation, one CTA pair per (query row, split)): a BF16 cache with bf16
  * operands; an E4M3 cache with f16 operands (the codes widened exactly, the
  * value rows multiplied by their scale once in f16, q_abs and the softmax
- * weights rounded to f16), so dequantised values must lie within f16's range.
+ * weights rounded to f16), so q_abs and the dequantised cache values must lie
+ * within f16's range (|x| <= 65504; a larger q_abs value would turn into an
+ * infinity and the scores of that query into NaN).
  * F32 runs exact fp32 on the CUDA cores.
+ * Concurrency: the tensor-core path hands out its work through a small
+ * counter that the library keys by o_part.  Calls that share o_part must not
+ * overlap on the GPU (they would also race on the partials); calls with
+ * different o_part buffers may run concurrently on different streams, as long
+ * as at most 64 distinct o_part buffers are in use at the same time.  A CUDA
+ * graph that captured this call keeps its o_part, so two replays of one graph
+ * must not overlap.
  * Pool contract: the tensor-core path reads whole 64-row pages.  Rows of a
  * sequence's last page beyond its length, and page 0 (read in place of a
  * block-table entry outside the pool), enter the contraction with zero
@@ -286,7 +295,9 @@ mla_status mla_out_uv(const void* o_lat, const void* w_uv, void* out, int rows, 
  *    every GPU that loads the library holds it until the process exits.
  *  - The first call on each device looks up the array's device address
  *    (cudaGetSymbolAddress, no allocation) with that device current; make
- *    that first call before any stream capture begins.
+ *    that first call before any stream capture begins.  The lookup is
+ *    repeated only if the device's context was replaced (cudaDeviceReset),
+ *    since the array then lives at a new address.
  *  - Every call uses the same array and it keeps the last call's contents.
  *    Each call writes every partial it reads before reading it, so nothing
  *    needs clearing.  Calls whose GPU work overlaps (on different streams,

@@ -34,9 +34,10 @@ _SIGS = {
     "mla_combine_shards": ("i", "ppiiipipp"),
     "mla_out_uv": ("i", "pppiiip"),
     "mla_decode_static": ("i", "pippiipiipiiiiifpippp"),
+    "mla_test_set_decode_wait": ("i", "Qi"),
 }
 _CT = {"p": ctypes.c_void_p, "i": ctypes.c_int, "f": ctypes.c_float, "d": ctypes.c_double,
-       "s": ctypes.c_char_p, "z": ctypes.c_size_t}
+       "s": ctypes.c_char_p, "z": ctypes.c_size_t, "Q": ctypes.c_ulonglong}
 
 _lib = None
 
@@ -181,5 +182,12 @@ def mla_decode_static(q_abs, q_dtype, cache, cache_scale, cache_dtype, num_pages
 
 
 MLA_STATIC_MAX_PARTIALS = 8192
+
+
+def mla_test_set_decode_wait(limit_cycles=0, withhold_q_load=False):
+    """Test hook (include/mla_test.h): bound of the decode kernel's barrier
+    waits in SM cycles (0 = the default) and whether the first query load of
+    every CTA pair is left out so that a wait runs out."""
+    _check("mla_test_set_decode_wait", lib().mla_test_set_decode_wait(int(limit_cycles), int(bool(withhold_q_load))))
 
 from .step import DecodeStep  # noqa: E402,F401

@@ -1,0 +1,672 @@
+// Split-KV latent attention for 65..128 heads over a bf16 cache, on the
+// tcgen05 tensor cores, with the heads split between the two CTAs of a pair.
+//
+// What it computes ("DeepSeek-V2: MLA Explained", "MLA Full Formulas" part 3
+// with the absorption of "Optimization Note"): for each head h of query row
+// r and each cached row j of the split that the query sees,
+//   z_j = scale * (q_abs[r,h,0:512] . c_j + q_abs[r,h,512:576] . k_j)
+// then the split's normalised softmax-weighted mean of the latents c_j and
+// its log-normaliser.
+//
+// How.  All heads share the cached rows, so both contractions are dense
+// GEMMs per tile of 256 rows, issued for the CTA pair (cta_group::2) with
+// M = 128 heads:
+//   S[128 heads x 256 rows]  = Q[128 x 576] . K[256 x 576]^T    (N = 256)
+//   O[128 heads x 512 dims] += P[128 x 256] . V[256 x 512]      (two MMAs of N = 256)
+// With M = 128 over a pair, CTA r holds heads [64r, 64r+64) of Q (the A
+// operand, 72 KB) and its TMEM receives S for those heads over all 256 rows
+// of the tile: lanes 0-63 hold the 128 rows that CTA 0 loaded (the B operand
+// is split by rows), lanes 64-127 the rows CTA 1 loaded.  The softmax of a
+// head therefore never needs the other CTA: each of its four threads (two
+// lane halves x two column halves) takes 64 scores, one page of the
+// sequence, and they combine maxima and sums through shared memory.  Each
+// thread writes its 64 probabilities as one 128-byte line of a K-major
+// [64 heads x 64 rows] bf16 tile, the A operand of the value MMA for that
+// page.  V is the B operand, split by dims: CTA r provides dims [128r,
+// 128r+128) and [256+128r, 256+128r+128) of every row of the tile; its own
+// rows come back from L2 (score loads are evict-last), the peer's rows were
+// read from HBM by the peer.  The value MMAs accumulate O in TMEM, 128 lanes
+// x 256 columns per CTA (lanes 0-63: the lower 128 dims of each 256-dim
+// half, lanes 64-127: the upper 128).
+//
+// Cache rows stream through a ring of seven 16 KB shared-memory stages
+// filled by TMA (128-byte swizzle) in the order the MMA consumes them: per
+// tile the nine score stages of tile i+1 follow the value stages of tile i,
+// so the score GEMM runs a tile ahead of the value GEMM and the softmax of a
+// tile overlaps the tensor work.  Pairs are persistent and claim (query
+// row, split) units dynamically.  Every barrier wait is bounded: on a
+// timeout the kernel flags MLA_DEVERR_TIMEOUT, lets its copies land, frees
+// its tensor memory and returns.
+//
+// Warp roles per CTA: 0 TMA producer and TMEM allocator, 1 MMA issuer (the
+// leader CTA issues for the pair), 2-9 softmax (warp w reads TMEM lanes
+// 32 (w % 4) .. +31; warps 2-5 take score columns 0-63, warps 6-9 64-127).
+#include <math.h>
+
+#include <mutex>
+
+#include "mla_device.cuh"
+#include "mla_internal.h"
+#include "sm100.cuh"
+
+namespace mla {
+namespace {
+
+using namespace sm100;
+
+constexpr int kTile = 256;                // cached rows per pair tile (128 per CTA)
+constexpr int kChunks = 9;                // 576 / 64 column chunks
+constexpr int kHPC = 64;                  // heads per CTA
+constexpr int kSlots = 7;                 // ring stages
+constexpr int kSlotBytes = 16384;         // one stage: one score chunk or one value box of this CTA
+constexpr int kBox = 8192;                // [64 rows x 64 bf16]
+constexpr int kQChunk = kHPC * 128;       // [64 heads x 64 dims] bf16
+constexpr int kPChunk = kHPC * 128;       // [64 heads x 64 rows] bf16: P of one page
+constexpr int kWarpProd = 0, kWarpMma = 1, kWarpSoft0 = 2, kSoftWarps = 8;
+constexpr int kThreads = 32 * (kWarpSoft0 + kSoftWarps);
+constexpr int kQN = 8;                    // unit queue depth
+constexpr float kRescaleLog2 = 8.0f;      // lazy rescale threshold (log2 units)
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 0;             // S of tile t at kColS + 128 (t & 1)
+constexpr uint32_t kColO = 256;           // O: dims 0..255 at 256, dims 256..511 at 384
+
+// shared memory (bytes from the 1024-aligned base)
+constexpr int kOffQ = 0;                                  // Q: 9 x 8 KB, K-major SW128
+constexpr int kOffRing = kOffQ + kChunks * kQChunk;       // ring: 7 x 16 KB
+constexpr int kOffP = kOffRing + kSlots * kSlotBytes;     // P: 4 pages x 8 KB, K-major SW128
+constexpr int kOffMisc = kOffP + 4 * kPChunk;
+constexpr int kMBars = 0;                 // 48 barriers
+constexpr int kMTmem = 48 * 8;
+constexpr int kMAbort = kMTmem + 4;
+constexpr int kMRedMax = kMTmem + 16;     // float [2 lane halves][2 column halves][64 heads]
+constexpr int kMRedSum = kMRedMax + 4 * kHPC * 4;
+constexpr int kMUnitQ = kMRedSum + 4 * kHPC * 4;
+constexpr int kMiscBytes = kMUnitQ + 4 * kQN;
+constexpr int kSmem = kOffMisc + kMiscBytes + 1024;       // + alignment slack
+static_assert(kSmem <= 227 * 1024, "shared memory budget");
+
+// barrier indices
+constexpr int kBFull = 0;                 // [kSlots] leader: both CTAs' TMA bytes of a stage
+constexpr int kBEmpty = kSlots;           // [kSlots] both: the MMAs are done with the stage
+constexpr int kBSFull = 2 * kSlots;       // [2] both: S of a tile is in TMEM
+constexpr int kBODone = kBSFull + 2;      // both: the value MMAs of a tile are done
+constexpr int kBPFull = kBODone + 1;      // leader: both CTAs' softmax wrote P (and rescaled O)
+constexpr int kBQFull = kBPFull + 1;      // leader: both CTAs' Q of the unit landed
+constexpr int kBQFree = kBQFull + 1;      // both: the unit's score MMAs are done with Q
+constexpr int kBEpiDone = kBQFree + 1;    // leader: both CTAs read O out (TMEM reusable)
+constexpr int kBUqFull = kBEpiDone + 1;   // [kQN] both: unit queue slot written
+constexpr int kBUqEmpty = kBUqFull + kQN; // [kQN] leader: every consumer read the slot
+constexpr int kBSoft = kBUqEmpty + kQN;   // [2] local: the softmax warps' own barriers (bounded waits)
+constexpr int kBEnd = kBSoft + 2;
+static_assert(kBEnd <= 48, "barrier area");
+
+struct PairParams {
+  int n_heads, q_len, batch;
+  const int32_t* block_table;
+  int max_pages, num_pages;
+  const int32_t* seq_lens;
+  int num_splits, split_tokens;
+  float scale_log2;            // softmax_scale * log2(e)
+  unsigned* claim;             // unit counter of this launch (0 at launch; reset by the last pair)
+  unsigned* done;              // pairs finished
+  float* o_part;
+  float* lse_part;
+  int32_t* err;
+  unsigned long long wait_limit;
+  int withhold_q;
+};
+
+// page id of a cached row of sequence b (0 for rows outside the table or the
+// pool: those rows are masked, and page 0 is readable memory)
+__device__ __forceinline__ int page_of(const PairParams& p, int b, int row, bool* ok) {
+  const int pidx = row >> 6;
+  int pg = -1;
+  if (pidx < p.max_pages) pg = p.block_table[(size_t)b * p.max_pages + pidx];
+  *ok = pg >= 0 && pg < p.num_pages;
+  return *ok ? pg : 0;
+}
+
+__device__ __forceinline__ void st_cluster_b32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    decode_pair_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_constant__ CUtensorMap tm_cache2,
+                       const __grid_constant__ CUtensorMap tm_q, const PairParams p) {
+  constexpr int kQConsumers = 2 + 2 * kSoftWarps;   // peer producer, MMA warp, softmax warps of both CTAs
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t s_base = smem_u32(smem);
+  const uint32_t s_q = s_base + kOffQ, s_ring = s_base + kOffRing;
+  uint8_t* misc = smem + kOffMisc;
+  const uint32_t s_misc = s_base + kOffMisc;
+  auto bar = [&](int i) -> uint32_t { return s_misc + kMBars + 8 * i; };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + kMAbort);
+  float* red_max = reinterpret_cast<float*>(misc + kMRedMax);
+  float* red_sum = reinterpret_cast<float*>(misc + kMRedSum);
+  int* unit_q = reinterpret_cast<int*>(misc + kMUnitQ);
+  uint8_t* s_pbuf = smem + kOffP;
+  const uint32_t s_p = s_base + kOffP;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint64_t lim = p.wait_limit;
+  const uint32_t rank = cluster_rank();
+  const uint32_t peer = rank ^ 1u;
+  const bool leader = rank == 0;
+
+  // ---- units: (query row r, split s), claimed by persistent pairs; every
+  // role walks the pair's same sequence, so barrier phases count globally
+  const int S = p.num_splits;
+  const int n_units = p.batch * p.q_len * S;
+  const int n_pairs = gridDim.x >> 1;
+  struct UnitInfo { int r, s, b, lo, hi, n_tiles; };
+  auto unit_at = [&](int u) -> UnitInfo {
+    UnitInfo x;
+    x.r = u / S;
+    x.s = u % S;
+    x.b = x.r / p.q_len;
+    const int t = x.r % p.q_len;
+    const int n_vis = p.seq_lens[x.b] - p.q_len + t + 1;
+    x.lo = x.s * p.split_tokens;
+    x.hi = min(x.lo + p.split_tokens, n_vis);
+    const int n_tok = x.hi - x.lo;
+    x.n_tiles = n_tok > 0 ? (n_tok + kTile - 1) / kTile : 0;
+    return x;
+  };
+
+  // ---- set-up
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kSlots; ++i) {
+      mbar_init(bar(kBFull + i), 1);
+      mbar_init(bar(kBEmpty + i), 1);
+    }
+    mbar_init(bar(kBSFull), 1);
+    mbar_init(bar(kBSFull + 1), 1);
+    mbar_init(bar(kBODone), 1);
+    mbar_init(bar(kBPFull), 2 * kSoftWarps);
+    mbar_init(bar(kBQFull), 1);
+    mbar_init(bar(kBQFree), 1);
+    mbar_init(bar(kBEpiDone), 2 * kSoftWarps);
+    for (int i = 0; i < kQN; ++i) {
+      mbar_init(bar(kBUqFull + i), 1);
+      mbar_init(bar(kBUqEmpty + i), kQConsumers);
+    }
+    mbar_init(bar(kBSoft), kSoftWarps);
+    mbar_init(bar(kBSoft + 1), kSoftWarps);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kWarpProd) tmem_alloc_pair(s_misc + kMTmem, kTmemCols);
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(misc + kMTmem);
+
+  // ---- the pair's unit sequence: the leader's producer claims units from the
+  // launch's counter and posts them, in order, to a queue in both CTAs
+  auto claim = [&](uint32_t k) -> int {      // leader producer, lane 0
+    const uint32_t slot = k % kQN;
+    if (k >= kQN && !mbar_wait(bar(kBUqEmpty + slot), ((k / kQN) - 1) & 1, abort_flag, lim)) return -2;
+    const unsigned cu = atomicAdd(p.claim, 1u);
+    const int uu = cu < (unsigned)n_units ? (int)cu : -1;
+    *reinterpret_cast<volatile int*>(unit_q + slot) = uu;
+    st_cluster_b32(mapa(smem_u32(unit_q + slot), peer), (uint32_t)uu);
+    mbar_arrive_cluster(bar(kBUqFull + slot));
+    mbar_arrive_cluster(mapa(bar(kBUqFull + slot), peer));
+    return uu;
+  };
+  auto next_unit = [&](uint32_t k) -> int {  // whole warp
+    const uint32_t slot = k % kQN;
+    if (!__all_sync(0xffffffffu, mbar_wait(bar(kBUqFull + slot), (k / kQN) & 1, abort_flag, lim))) return -2;
+    const int uu = *reinterpret_cast<volatile int*>(unit_q + slot);
+    __syncwarp();
+    if (lane == 0) mbar_arrive_cluster(mapa(bar(kBUqEmpty + slot), 0));
+    return uu;
+  };
+
+  uint32_t kc = 0;   // ring stages handed out (producer) or consumed (MMA)
+  if (warp == kWarpProd) {
+    // ============ TMA producer (both CTAs), in the order the MMA consumes ============
+    // S(0), then per tile i: S(i+1), O(i).  The pool is page-blocked (nine
+    // contiguous [64 rows x 64 columns] blocks per page), viewed as 2-D
+    // [blocks * 64 lines x 64 columns].  A score stage is column chunk c of
+    // this CTA's two pages of the tile (lane l < 2: block c of page l, 8 KB);
+    // a value stage is one page's pair of dims blocks 4 bb + 2 r, +1 of this
+    // CTA (one contiguous 16 KB box).
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_cache);
+      tma_prefetch_desc(&tm_cache2);
+      tma_prefetch_desc(&tm_q);
+    }
+    auto take = [&](uint32_t bytes, uint32_t& dst, uint32_t& fb) -> bool {
+      const uint32_t slot = kc % kSlots;
+      const uint32_t ph = (kc / kSlots) & 1u;
+      bool ok = true;
+      if (lane == 0) {
+        ok = mbar_wait<false>(bar(kBEmpty + slot), ph ^ 1u, abort_flag, lim);
+        if (ok && leader) mbar_arrive_expect_tx(bar(kBFull + slot), 2u * bytes);
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      dst = s_ring + slot * kSlotBytes;
+      fb = mapa(bar(kBFull + slot), 0);
+      ++kc;
+      return ok;
+    };
+    // score rows are re-read by the value stages of the pair (this CTA's for
+    // its dims, the peer's for the other dims) one tile later: evict-last;
+    // value loads are the rows' last use: evict-first
+    const uint64_t pol_keep = policy_evict_last();
+    const uint64_t pol_drop = policy_evict_first();
+    uint32_t uc = 0;
+    bool ok = true;
+    for (uint32_t k = 0; ok; ++k) {
+      int u;
+      if (leader) {
+        int uu = 0;
+        if (lane == 0) uu = claim(k);
+        u = __shfl_sync(0xffffffffu, uu, 0);
+      } else {
+        u = next_unit(k);
+      }
+      if (u == -2) { ok = false; break; }
+      if (u < 0) break;
+      const UnitInfo U = unit_at(u);
+      if (U.n_tiles == 0) continue;
+      const int r = U.r, b = U.b, lo = U.lo, hi = U.hi, n_tiles = U.n_tiles;
+      if (lane == 0) {
+        // the previous unit's score MMAs must be done with Q (both halves)
+        if (uc > 0) ok = mbar_wait<false>(bar(kBQFree), (uc - 1) & 1, abort_flag, lim);
+        // (test hook: the leader leaves the query load of its first unit out,
+        // so the MMA issuer's wait for it runs out and the launch aborts)
+        if (ok && !(p.withhold_q && leader && uc == 0)) {
+          const uint32_t q_bar = mapa(bar(kBQFull), 0);
+          if (leader) mbar_arrive_expect_tx(bar(kBQFull), 2u * kChunks * kQChunk);
+          for (int c = 0; c < kChunks; ++c)
+            tma_load_3d_pair(s_q + c * kQChunk, &tm_q, 64 * c, (int)rank * kHPC, r, q_bar);
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      auto load_s = [&](int i) -> bool {
+        bool vv;
+        const int pg = page_of(p, b, lo + kTile * i + 128 * (int)rank + 64 * (lane & 1), &vv);
+        for (int c = 0; c < kChunks; ++c) {
+          uint32_t dst, fb;
+          if (!take(kSlotBytes, dst, fb)) return false;
+          if (lane < 2) tma_load_2d_pair_hint(dst + lane * kBox, &tm_cache, 0, (pg * kChunks + c) * 64, fb, pol_keep);
+        }
+        return true;
+      };
+      auto load_o = [&](int j) -> bool {
+        for (int pg_i = 0; pg_i < 4; ++pg_i) {
+          const int row0 = lo + kTile * j + 64 * pg_i;
+          if (row0 >= hi) break;
+          bool vld;
+          const int pg = page_of(p, b, row0, &vld);
+          for (int bb = 0; bb < 2; ++bb) {
+            uint32_t dst, fb;
+            if (!take(kSlotBytes, dst, fb)) return false;
+            if (lane == 0)
+              tma_load_2d_pair_hint(dst, &tm_cache2, 0, (pg * kChunks + 4 * bb + 2 * (int)rank) * 64, fb, pol_drop);
+          }
+        }
+        return true;
+      };
+      ok = load_s(0);
+      for (int i = 0; i < n_tiles && ok; ++i) {
+        if (i + 1 < n_tiles) ok = load_s(i + 1);
+        if (ok) ok = load_o(i);
+      }
+      ++uc;
+    }
+  } else if (warp == kWarpMma) {
+    // ================= MMA issuer (leader CTA, whole warp, one elected lane) =================
+    // Per unit: S(0), then per tile i: S(i+1), O(i).  S(i+1) goes to the
+    // other TMEM buffer while the softmax of tile i reads S(i); S(i+2) reuses
+    // S(i)'s columns after O(i), which waited for the softmax of tile i.
+    if (leader) {
+      constexpr uint32_t idS = idesc_f16(128, 256, false, false);
+      constexpr uint32_t idO = idesc_f16(128, 256, false, true);
+      auto ready = [&](uint32_t& src, uint32_t& empty) -> bool {
+        const uint32_t slot = kc % kSlots;
+        const uint32_t ph = (kc / kSlots) & 1u;
+        if (!__all_sync(0xffffffffu, mbar_wait<false>(bar(kBFull + slot), ph, abort_flag, lim))) return false;
+        tc_fence_after();
+        src = s_ring + slot * kSlotBytes;
+        empty = bar(kBEmpty + slot);
+        ++kc;
+        return true;
+      };
+      uint32_t uc = 0, gt = 0;
+      bool ok = true;
+      for (uint32_t k = 0; ok; ++k) {
+        const int u = next_unit(k);
+        if (u == -2) { ok = false; break; }
+        if (u < 0) break;
+        const UnitInfo U = unit_at(u);
+        if (U.n_tiles == 0) continue;
+        const int lo = U.lo, hi = U.hi, n_tiles = U.n_tiles;
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(kBQFull), uc & 1, abort_flag, lim));
+        if (!ok) break;
+        tc_fence_after();
+        auto issue_s = [&](int i) -> bool {
+          const uint32_t sb = (gt + i) & 1u;
+          const uint32_t d = tmem + kColS + 128 * sb;
+          const uint64_t qd = smem_desc_sw128(s_q, 16, 1024);
+          for (int c = 0; c < kChunks; ++c) {
+            uint32_t a0, empty;
+            if (!ready(a0, empty)) return false;
+            const uint64_t kd = smem_desc_sw128(a0, 16, 1024);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)   // K = 16 per MMA: +32 bytes along the 128-byte lines
+              mma_pair_f16_w(d, qd + ((c * kQChunk + ks * 32) >> 4), kd + ((ks * 32) >> 4), idS, (c | ks) != 0);
+            mma_commit_pair_w(empty, 0x3);
+          }
+          mma_commit_pair_w(bar(kBSFull + sb), 0x3);
+          // the unit's last score GEMM: Q may be replaced once it completes
+          if (i == n_tiles - 1) mma_commit_pair_w(bar(kBQFree), 0x3);
+          return true;
+        };
+        auto issue_o = [&](int j) -> bool {
+          const uint32_t t = gt + j;
+          if (!__all_sync(0xffffffffu, mbar_wait(bar(kBPFull), t & 1, abort_flag, lim))) return false;
+          // the accumulator is overwritten by this unit's first value MMA: the
+          // previous unit's epilogue must have read it out
+          if (j == 0 && uc > 0 &&
+              !__all_sync(0xffffffffu, mbar_wait(bar(kBEpiDone), (uc - 1) & 1, abort_flag, lim)))
+            return false;
+          tc_fence_after();
+          const uint64_t pd = smem_desc_sw128(s_p, 16, 1024);
+          for (int pg_i = 0; pg_i < 4; ++pg_i) {
+            if (lo + kTile * j + 64 * pg_i >= hi) break;
+            for (int bb = 0; bb < 2; ++bb) {
+              uint32_t b0, empty;
+              if (!ready(b0, empty)) return false;
+              const uint64_t vd = smem_desc_sw128(b0, kBox, 1024);
+#pragma unroll
+              for (int ks = 0; ks < 4; ++ks)   // 16 rows per MMA: +32 bytes of P lines, +2 KB of V lines
+                mma_pair_f16_w(tmem + kColO + 128 * bb, pd + ((pg_i * kPChunk + ks * 32) >> 4),
+                               vd + ((ks * 2048) >> 4), idO, (j | pg_i | ks) != 0);
+              mma_commit_pair_w(empty, 0x3);
+            }
+          }
+          mma_commit_pair_w(bar(kBODone), 0x3);
+          return true;
+        };
+        ok = issue_s(0);
+        for (int i = 0; i < n_tiles && ok; ++i) {
+          if (i + 1 < n_tiles) ok = issue_s(i + 1);
+          if (ok) ok = issue_o(i);
+        }
+        gt += n_tiles;
+        ++uc;
+      }
+    }
+  } else {
+    // ================= softmax (both CTAs, warps 2-9) =================
+    // Thread (lane quadrant q4, column half ch, lane) owns head hh = 32 (q4 & 1)
+    // + lane of this CTA and the 64 tile rows 128 (q4 >> 1) + 64 ch .. +63.
+    const int q4 = warp & 3;
+    const int half = q4 >> 1;                   // 0: TMEM lanes 0-63, 1: lanes 64-127
+    const int hh = 32 * (q4 & 1) + lane;        // head within this CTA
+    const int head = kHPC * (int)rank + hh;
+    const int ch = (warp - kWarpSoft0) >> 2;    // score columns [64 ch, 64 ch + 64)
+    const uint32_t lane_addr = static_cast<uint32_t>(32 * q4) << 16;
+    const int part = 2 * half + ch;             // which of the head's four partial results (= page of the tile)
+    // barriers among the eight softmax warps, on mbarriers so that every wait
+    // is bounded: a warp that leaves on a timeout cannot strand the others
+    uint32_t soft_ph[2] = {0, 0};
+    auto soft_sync = [&](int which) -> bool {
+      __syncwarp();
+      if (lane == 0) mbar_arrive_local(bar(kBSoft + which));
+      const bool okk = __all_sync(0xffffffffu, mbar_wait<false>(bar(kBSoft + which), soft_ph[which] & 1,
+                                                                abort_flag, lim));
+      ++soft_ph[which];
+      return okk;
+    };
+    uint32_t uc = 0, gt = 0;
+    bool ok = true;
+    for (uint32_t k = 0; ok; ++k) {
+      const int u = next_unit(k);
+      if (u == -2) { ok = false; break; }
+      if (u < 0) break;
+      const UnitInfo U = unit_at(u);
+      const int r = U.r, s = U.s, b = U.b, lo = U.lo, hi = U.hi, n_tiles = U.n_tiles;
+      if (n_tiles == 0) {
+        // nothing visible in this split: lse = -inf; o_part is left unwritten
+        // (the merge gives such a split weight 0 and does not read it)
+        if (part == 0 && head < p.n_heads) p.lse_part[((size_t)r * p.n_heads + head) * S + s] = -INFINITY;
+        continue;
+      }
+      float m_run = -INFINITY, l_acc = 0.f;
+      for (int i = 0; i < n_tiles; ++i) {
+        const uint32_t t = gt + i;
+        const uint32_t sb = t & 1u;
+        ok = __all_sync(0xffffffffu, mbar_wait<false>(bar(kBSFull + sb), (t >> 1) & 1, abort_flag, lim));
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t scol = tmem + lane_addr + kColS + 128 * sb;
+        float v[64];
+        tmem_ld<32>(scol + 64 * ch, v);
+        tmem_ld<32>(scol + 64 * ch + 32, v + 32);
+        tmem_wait_ld();
+        // rows of this thread: one page of the sequence
+        const int row0 = lo + kTile * i + 128 * half + 64 * ch;
+        int nvalid = min(max(hi - row0, 0), 64);
+        if (nvalid > 0) {
+          bool pok;
+          (void)page_of(p, b, row0, &pok);
+          if (!pok) {
+            nvalid = 0;
+            flag_error(p.err, MLA_DEVERR_PAGE);
+          }
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < 64; ++j) {
+          v[j] = j < nvalid ? v[j] * p.scale_log2 : -INFINITY;
+          mx = fmaxf(mx, v[j]);
+        }
+        red_max[part * kHPC + hh] = mx;
+        if (!(ok = soft_sync(0))) break;
+        const float tmax = fmaxf(fmaxf(red_max[hh], red_max[kHPC + hh]),
+                                 fmaxf(red_max[2 * kHPC + hh], red_max[3 * kHPC + hh]));
+        const float m_new = (tmax > m_run + kRescaleLog2) ? tmax : m_run;
+        const bool changed = m_new != m_run;
+        // factor for the sums and the accumulator kept so far (0 when nothing was kept)
+        const float alpha = (m_run == -INFINITY) ? 0.f : exp2_approx(m_run - m_new);
+        m_run = m_new;
+        const float msub = m_new == -INFINITY ? 0.f : m_new;
+        uint32_t pk[32];
+        float sum = 0.f;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const float p0 = exp2_approx(v[2 * j] - msub), p1 = exp2_approx(v[2 * j + 1] - msub);
+          sum += p0 + p1;
+          pk[j] = pack_bf16(p0, p1);
+        }
+        l_acc = changed ? fmaf(l_acc, alpha, sum) : l_acc + sum;
+        // every phase of o_done is observed in order (a parity wait cannot
+        // tell a phase two behind from a completed one); O(i-1) done also
+        // frees the P tiles for this tile's probabilities
+        if (i >= 1) {
+          ok = __all_sync(0xffffffffu, mbar_wait<false>(bar(kBODone), (t - 1) & 1, abort_flag, lim));
+          if (!ok) break;
+          tc_fence_after();
+          if (__any_sync(0xffffffffu, changed)) {
+            const float f = changed ? alpha : 1.f;
+            const uint32_t oc = tmem + lane_addr + kColO + 128 * ch;
+#pragma unroll 1
+            for (int c4 = 0; c4 < 4; ++c4) {
+              float o[32];
+              tmem_ld<32>(oc + 32 * c4, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int j = 0; j < 32; ++j) o[j] *= f;
+              tmem_st<32>(oc + 32 * c4, o);
+            }
+          }
+        }
+        // P of this thread's 64 rows (one page of the tile): line hh of the
+        // page's K-major [64 heads x 64 rows] tile, 128-byte swizzled
+        {
+          uint8_t* line = s_pbuf + part * kPChunk + hh * 128;
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            *reinterpret_cast<uint4*>(line + ((q ^ (hh & 7)) << 4)) =
+                make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        }
+        fence_proxy_async_cta();     // read by the tensor core
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(mapa(bar(kBPFull), 0));
+      }
+      // ---- epilogue: normalise O by the row sums, write o_part and lse
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait<false>(bar(kBODone), (gt + n_tiles - 1) & 1, abort_flag, lim));
+      if (ok) {
+        tc_fence_after();
+        red_sum[part * kHPC + hh] = l_acc;
+        ok = soft_sync(0);
+      }
+      if (ok) {
+        const float lt = red_sum[hh] + red_sum[kHPC + hh] + red_sum[2 * kHPC + hh] + red_sum[3 * kHPC + hh];
+        const float inv_l = lt > 0.f ? 1.0f / lt : 0.f;
+        const bool live = head < p.n_heads;
+        if (part == 0 && live)
+          p.lse_part[((size_t)r * p.n_heads + head) * S + s] =
+              lt > 0.f ? (m_run + log2f(lt)) * 0.69314718055994531f : -INFINITY;
+        // this thread's O: dims 256 ch + 128 half + (0..127) of head `head`
+        float* op = p.o_part + (((size_t)r * p.n_heads + head) * S + s) * MLA_D_C + 256 * ch + 128 * half;
+        const uint32_t oc = tmem + lane_addr + kColO + 128 * ch;
+#pragma unroll 1
+        for (int c4 = 0; c4 < 4; ++c4) {
+          float o[32];
+          tmem_ld<32>(oc + 32 * c4, o);
+          tmem_wait_ld();
+          if (live) {
+            float4* dst = reinterpret_cast<float4*>(op + 32 * c4);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              dst[j] = make_float4(o[4 * j] * inv_l, o[4 * j + 1] * inv_l, o[4 * j + 2] * inv_l, o[4 * j + 3] * inv_l);
+          }
+        }
+        // this warp's part of O has been read: the pair's next unit may overwrite it
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(mapa(bar(kBEpiDone), 0));
+      }
+      gt += n_tiles;
+      ++uc;
+    }
+  }
+
+  // ---- teardown
+  if (*abort_flag) {
+    if (threadIdx.x == 0) flag_error(p.err, MLA_DEVERR_TIMEOUT);
+    // let copies and MMAs already in flight land before the memory is released
+    const uint64_t t0 = globaltimer();
+    while (globaltimer() - t0 < 2000000ull) {
+    }
+  }
+  // the last pair to finish resets the launch's unit counter for the next launch
+  if (leader && threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(p.done, 1u) == (unsigned)(n_pairs - 1)) {
+      atomicExch(p.claim, 0u);
+      atomicExch(p.done, 0u);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  if (warp == kWarpProd) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+// Unit counters, one (claim, done) pair per launch in flight, keyed by the
+// launch's o_part workspace (see the decode_tc.cu counterpart for the rule).
+constexpr int kCounterSlots = 64;
+__device__ unsigned g_pair_claim[kCounterSlots];
+__device__ unsigned g_pair_done[kCounterSlots];
+
+bool claim_slot(const void* workspace, unsigned** claim, unsigned** done) {
+  static std::mutex mu;
+  static const void* owner[kCounterSlots] = {};
+  static unsigned next = 0;
+  void* c = nullptr;
+  void* d = nullptr;
+  if (cudaGetSymbolAddress(&c, g_pair_claim) != cudaSuccess || cudaGetSymbolAddress(&d, g_pair_done) != cudaSuccess)
+    return false;
+  unsigned i = kCounterSlots;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    for (unsigned k = 0; k < (unsigned)kCounterSlots; ++k)
+      if (owner[k] == workspace) { i = k; break; }
+    if (i == (unsigned)kCounterSlots) {
+      i = next++ % kCounterSlots;
+      owner[i] = workspace;
+    }
+  }
+  *claim = static_cast<unsigned*>(c) + i;
+  *done = static_cast<unsigned*>(d) + i;
+  return true;
+}
+
+}  // namespace
+
+bool decode_pair_supported(const DecodeArgs& a) {
+  return a.q_dtype == MLA_BF16 && a.cache_dtype == MLA_BF16 && a.page_size == 64 && a.n_heads > 64 &&
+         a.n_heads <= 128 && (long long)a.batch * a.q_len * a.num_splits * 2 < (1ll << 31);
+}
+
+cudaError_t launch_decode_pair(const DecodeArgs& a, cudaStream_t st) {
+  TensorMapEncodeFn enc = tensor_map_encoder();
+  if (!enc) return cudaErrorNotSupported;
+  CUtensorMap tc, tc2, tq;
+  // the page-blocked pool as 2-D [num_pages * 9 * 64 lines x 64 columns] of
+  // 128-byte lines: boxes of 64 lines (one block) and 128 lines (two adjacent blocks)
+  for (int k = 0; k < 2; ++k) {
+    cuuint64_t dims[2] = {64, (cuuint64_t)a.num_pages * kChunks * 64};
+    cuuint64_t strides[1] = {128};
+    cuuint32_t box[2] = {64, k == 0 ? 64u : 128u};
+    cuuint32_t es[2] = {1, 1};
+    if (enc(k == 0 ? &tc : &tc2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a.cache), dims, strides, box,
+            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  {
+    // q_abs [rows, heads, 576]: boxes of 64 columns x 64 heads of one row
+    // (heads past n_heads read as zeros)
+    cuuint64_t dims[3] = {MLA_D_ROW, (cuuint64_t)a.n_heads, (cuuint64_t)a.batch * a.q_len};
+    cuuint64_t strides[2] = {MLA_D_ROW * 2, (cuuint64_t)a.n_heads * MLA_D_ROW * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)kHPC, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    if (enc(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(a.q_abs), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  cudaError_t e = cudaFuncSetAttribute(decode_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+  if (e != cudaSuccess) return e;
+  PairParams p{a.n_heads, a.q_len, a.batch, a.block_table, a.max_pages, a.num_pages, a.seq_lens, a.num_splits,
+               a.split_tokens, a.softmax_scale * 1.4426950408889634f, nullptr, nullptr, a.o_part, a.lse_part, a.err,
+               g_wait_limit.load(), g_withhold_q.load()};
+  if (!claim_slot(a.o_part, &p.claim, &p.done)) return cudaErrorInvalidSymbol;
+  const long long units = (long long)a.batch * a.q_len * a.num_splits;
+  const long long P = sm_pair_count();
+  const long long pairs = units < P ? units : P;
+  decode_pair_kernel<<<dim3((unsigned)(2 * pairs)), kThreads, kSmem, st>>>(tc, tc2, tq, p);
+  return cudaGetLastError();
+}
+
+}  // namespace mla

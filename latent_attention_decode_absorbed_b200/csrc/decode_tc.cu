@@ -49,6 +49,7 @@
 #include <math.h>
 
 #include <atomic>
+#include <mutex>
 
 #include "mla_device.cuh"
 #include "mla_internal.h"
@@ -95,6 +96,8 @@ struct TcParams {
   float* o_part;
   float* lse_part;
   int32_t* err;
+  unsigned long long wait_limit;   // SM cycles a barrier wait may take before the launch aborts
+  int withhold_q;                  // test hook: the leader leaves its first unit's query load out
 };
 
 template <int NH, bool F8>
@@ -266,6 +269,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
   float* l_x = reinterpret_cast<float*>(misc + LY::kLX);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint64_t lim = p.wait_limit;
   const uint32_t rank = cluster_rank();
   const uint32_t peer = rank ^ 1u;
   const bool leader = rank == 0;
@@ -338,7 +342,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
   int* unit_q = reinterpret_cast<int*>(misc + LY::kUnitQ);
   auto claim = [&](uint32_t k) -> int {      // leader producer, lane 0
     const uint32_t slot = k % kQN;
-    if (k >= kQN && !mbar_wait(bar(B::uq_empty + slot), ((k / kQN) - 1) & 1, abort_flag)) return -2;
+    if (k >= kQN && !mbar_wait(bar(B::uq_empty + slot), ((k / kQN) - 1) & 1, abort_flag, lim)) return -2;
     const unsigned cu = atomicAdd(p.claim, 1u);
     const int uu = cu < (unsigned)n_units ? (int)cu : -1;
     *reinterpret_cast<volatile int*>(unit_q + slot) = uu;
@@ -349,7 +353,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
   };
   auto next_unit = [&](uint32_t k, bool whole_warp) -> int {
     const uint32_t slot = k % kQN;
-    if (!mbar_wait(bar(B::uq_full + slot), (k / kQN) & 1, abort_flag)) return -2;
+    if (!mbar_wait(bar(B::uq_full + slot), (k / kQN) & 1, abort_flag, lim)) return -2;
     const int uu = *reinterpret_cast<volatile int*>(unit_q + slot);
     if (whole_warp) __syncwarp();
     if (lane == 0) mbar_arrive_cluster(mapa(bar(B::uq_empty + slot), 0));
@@ -371,7 +375,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
     const uint32_t ph = (rg.kc / rg.slots) & 1u;
     bool ok = true;
     if (lane == 0) {
-      ok = mbar_wait<false>(rg.empty0 + 8 * slot, ph ^ 1u, abort_flag);
+      ok = mbar_wait<false>(rg.empty0 + 8 * slot, ph ^ 1u, abort_flag, lim);
       if (ok && leader) mbar_arrive_expect_tx(rg.full0 + 8 * slot, 2u * bytes);
     }
     ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -385,7 +389,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
     const uint32_t slot = rg.kc % rg.slots;
     const uint32_t ph = (rg.kc / rg.slots) & 1u;
     // e4m3: the converters arrive after generic-proxy writes (cluster scope)
-    if (!mbar_wait<F8>(rg.full0 + 8 * slot, ph, abort_flag)) return false;
+    if (!__all_sync(0xffffffffu, mbar_wait<F8>(rg.full0 + 8 * slot, ph, abort_flag, lim))) return false;
     tc_fence_after();
     src = rg.base + slot * kSlotBytes;
     empty = rg.empty0 + 8 * slot;
@@ -407,7 +411,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
         const uint32_t ph = (kc / LY::kSlots) & 1u;
         bool ok = true;
         if (lane == 0) {
-          ok = mbar_wait<false>(bar(B::sempty8 + slot), ph ^ 1u, abort_flag);
+          ok = mbar_wait<false>(bar(B::sempty8 + slot), ph ^ 1u, abort_flag, lim);
           if (ok) mbar_arrive_expect_tx(bar(B::sfull8 + slot), nbox * kBox8);
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -431,8 +435,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
       const int r = U.r, b = U.b, lo = U.lo, hi = U.hi, n_tiles = U.n_tiles;
       if (lane == 0) {
         // the previous unit's score MMAs must be done with Q
-        if (uc > 0) ok = mbar_wait<false>(bar(B::q_free), (uc - 1) & 1, abort_flag);
-        if (ok) {
+        if (uc > 0) ok = mbar_wait<false>(bar(B::q_free), (uc - 1) & 1, abort_flag, lim);
+        if (ok && !(p.withhold_q && leader && uc == 0)) {
           mbar_arrive_expect_tx(bar(B::q_full), kChunks * LY::kQChunk);
           for (int c = 0; c < kChunks; ++c)
             tma_load_3d(s_q + c * LY::kQChunk, &tm_q, 64 * c, (int)rank * HPW, r, bar(B::q_full));
@@ -496,7 +500,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
       const UnitInfo U = unit_at(u);
       if (U.n_tiles == 0) continue;
       const int b = U.b, lo = U.lo, hi = U.hi, n_tiles = U.n_tiles;
-      ok = __all_sync(0xffffffffu, mbar_wait<false>(bar(B::q_full), uc & 1, abort_flag));
+      ok = __all_sync(0xffffffffu, mbar_wait<false>(bar(B::q_full), uc & 1, abort_flag, lim));
       if (ok) {
         for (int i = ct; i < kChunks * LY::kQChunk / 16; i += kCT) {
           uint4 v = *reinterpret_cast<const uint4*>(smem + LY::kQ + 16 * i);
@@ -523,8 +527,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
         const uint32_t slot = kc % LY::kSlots;
         const uint32_t ph = (kc / LY::kSlots) & 1u;
         ++kc;
-        if (!__all_sync(0xffffffffu, mbar_wait<false>(bar(B::sfull8 + slot), ph, abort_flag))) return false;
-        if (!__all_sync(0xffffffffu, mbar_wait<false>(bar(B::empty + slot), ph ^ 1u, abort_flag))) return false;
+        if (!__all_sync(0xffffffffu, mbar_wait<false>(bar(B::sfull8 + slot), ph, abort_flag, lim))) return false;
+        if (!__all_sync(0xffffffffu, mbar_wait<false>(bar(B::empty + slot), ph ^ 1u, abort_flag, lim))) return false;
         const uint8_t* src = smem + LY::kStaging + slot * kStage8;
         uint8_t* dst = smem + LY::kRing + slot * kSlotBytes;
         // 16 codes (one quarter of a 64-byte row) per step
@@ -608,8 +612,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
     const int r = U.r, b = U.b, lo = U.lo, hi = U.hi, n_tiles = U.n_tiles;
     if (lane == 0) {
       // the previous unit's score MMAs must be done with Q (both halves)
-      if (uc > 0) ok = mbar_wait<false>(bar(B::q_free), (uc - 1) & 1, abort_flag);
-      if (ok) {
+      if (uc > 0) ok = mbar_wait<false>(bar(B::q_free), (uc - 1) & 1, abort_flag, lim);
+      // (test hook: the leader leaves the query load of its first unit out, so
+      // the MMA issuer's wait for it runs out and the launch aborts cleanly)
+      if (ok && !(p.withhold_q && leader && uc == 0)) {
         const uint32_t q_bar = mapa(bar(B::q_full), 0);
         if (leader) mbar_arrive_expect_tx(bar(B::q_full), 2u * kChunks * LY::kQChunk);
         for (int c = 0; c < kChunks; ++c)
@@ -671,27 +677,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
     // warps read the previous unit's O^T out; its first O^T MMA waits for that.
     // Tiles are numbered globally (gt + i) for the S^T buffers, the P^T ring
     // and the per-tile barriers.
-    if (leader && lane == 0) {
+    if (leader) {
       // e4m3 cache: the operands are f16 (widened codes, Q and P in f16)
       constexpr uint32_t idS = idesc_f16(256, NH, false, false, F8);
       constexpr uint32_t idO = idesc_f16(256, NH, true, false, F8);
       uint32_t uc = 0, gt = 0;
       bool ok = true;
       for (uint32_t k = 0; ok; ++k) {
-      const int u = next_unit(k, false);
+      const int u = next_unit(k, true);
       if (u == -2) { ok = false; break; }
       if (u < 0) break;
       const UnitInfo U = unit_at(u);
       if (U.n_tiles == 0) continue;
       const int lo = U.lo, hi = U.hi, n_tiles = U.n_tiles;
-      ok = mbar_wait(bar(F8 ? B::q_ready : B::q_full), uc & 1, abort_flag);
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(F8 ? B::q_ready : B::q_full), uc & 1, abort_flag, lim));
       if (!ok) break;
       tc_fence_after();
       auto issue_s = [&](int i) -> bool {
         const uint32_t gi = gt + i;
         const int sb = gi & 1;
         if (gi >= 2) {
-          if (!mbar_wait(bar(B::s_free + sb), ((gi - 2) >> 1) & 1, abort_flag)) return false;
+          if (!__all_sync(0xffffffffu, mbar_wait(bar(B::s_free + sb), ((gi - 2) >> 1) & 1, abort_flag, lim))) return false;
           tc_fence_after();
         }
         const uint32_t d = tmem + (sb ? kColS1 : kColS0);
@@ -705,22 +711,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
             for (int ks = 0; ks < 4; ++ks) {
               const uint64_t ad = smem_desc_sw128(a0 + cc * kChunkBytes + ks * 32, 16, 1024);
               const uint64_t bd = smem_desc_sw128(s_q + c * LY::kQChunk + ks * 32, 16, 1024);
-              mma_pair_f16(d, ad, bd, idS, (c | ks) != 0);
+              mma_pair_f16_w(d, ad, bd, idS, (c | ks) != 0);
             }
           }
-          mma_commit_pair(empty, 0x3);
+          mma_commit_pair_w(empty, 0x3);
         }
-        mma_commit_pair(bar(B::s_full + sb), 0x3);
+        mma_commit_pair_w(bar(B::s_full + sb), 0x3);
         // the unit's last score GEMM: Q may be replaced once it completes
-        if (i == n_tiles - 1) mma_commit_pair(bar(B::q_free), 0x3);
+        if (i == n_tiles - 1) mma_commit_pair_w(bar(B::q_free), 0x3);
         return true;
       };
       auto issue_o = [&](int j) -> bool {
         const uint32_t gj = gt + j;
-        if (!mbar_wait(bar(B::p_full), gj & 1, abort_flag)) return false;
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(B::p_full), gj & 1, abort_flag, lim))) return false;
         // the accumulator is overwritten by this unit's first O^T MMA: the
         // previous unit's epilogue must have read it out
-        if (j == 0 && uc > 0 && !mbar_wait(bar(B::epi_done), (uc - 1) & 1, abort_flag)) return false;
+        if (j == 0 && uc > 0 && !__all_sync(0xffffffffu, mbar_wait(bar(B::epi_done), (uc - 1) & 1, abort_flag, lim))) return false;
         tc_fence_after();
         for (int pg_i = 0; pg_i < 4; ++pg_i) {
           // P^T chunk pg_i of global tile gj lives in slot (4 gj + pg_i) mod
@@ -734,14 +740,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
               for (int ks = 0; ks < 4; ++ks) {
                 const uint64_t ad = smem_desc_sw128(a0 + bb * kChunkBytes + ks * 2048, kBoxBytes, 1024);
                 const uint64_t bd = smem_desc_sw128(s_p + pslot * LY::kPChunk + ks * 32, 16, 1024);
-                mma_pair_f16(tmem + kColO + bb * 128, ad, bd, idO, (j | pg_i | ks) != 0);
+                mma_pair_f16_w(tmem + kColO + bb * 128, ad, bd, idO, (j | pg_i | ks) != 0);
               }
             }
-            mma_commit_pair(empty, 0x3);
+            mma_commit_pair_w(empty, 0x3);
           }
-          mma_commit_pair(bar(B::p_free + pslot), 0x3);
+          mma_commit_pair_w(bar(B::p_free + pslot), 0x3);
         }
-        mma_commit_pair(bar(B::o_done), 0x3);
+        mma_commit_pair_w(bar(B::o_done), 0x3);
         return true;
       };
       ok = issue_s(0);
@@ -805,7 +811,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
     for (int i = 0; i < n_tiles; ++i) {
       const uint32_t gi = gt + i;              // global tile number: buffers and phases
       const int sb = gi & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait<false>(bar(B::s_full + sb), (gi >> 1) & 1, abort_flag));
+      ok = __all_sync(0xffffffffu, mbar_wait<false>(bar(B::s_full + sb), (gi >> 1) & 1, abort_flag, lim));
       if (!ok) break;
       tc_fence_after();
       const int row = lo + kTile * i + kt;
@@ -859,7 +865,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
           own_max[g * HPG + h] = tm;
           st_async_f32(mapa(smem_u32(x_max + xb * NH + g * HPG + h), peer), tm, peer_bar);
         }
-        if (__all_sync(0xffffffffu, mbar_wait(bar(B::mx_full + xb), (gi >> 1) & 1, abort_flag))) {
+        if (__all_sync(0xffffffffu, mbar_wait(bar(B::mx_full + xb), (gi >> 1) & 1, abort_flag, lim))) {
           int ch = 0;
           for (int h = lane; h < HPG; h += 32) {
             const float mt = fmaxf(own_max[g * HPG + h], x_max[xb * NH + g * HPG + h]);
@@ -893,12 +899,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
       const int pslot = pn % LY::kPSlots;
       if (pn >= LY::kPSlots) {
         ok = __all_sync(0xffffffffu,
-                        mbar_wait<false>(bar(B::p_free + pslot), ((pn / LY::kPSlots) - 1) & 1, abort_flag));
+                        mbar_wait<false>(bar(B::p_free + pslot), ((pn / LY::kPSlots) - 1) & 1, abort_flag, lim));
         if (!ok) break;
       }
       const uint32_t row_base = pslot * LY::kPChunk + (wcol & 7) * 2;
       if (i >= 1) {
-        ok = __all_sync(0xffffffffu, mbar_wait<false>(bar(B::o_done), (gi - 1) & 1, abort_flag));
+        ok = __all_sync(0xffffffffu, mbar_wait<false>(bar(B::o_done), (gi - 1) & 1, abort_flag, lim));
         if (!ok) break;
         tc_fence_after();
       }
@@ -952,7 +958,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
       if (lane == 0) mbar_arrive_cluster(mapa(bar(B::p_full), 0));
     }
     // ---- epilogue: normalise O^T by the row sums, write o_part and lse
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait<false>(bar(B::o_done), (gt + n_tiles - 1) & 1, abort_flag));
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait<false>(bar(B::o_done), (gt + n_tiles - 1) & 1, abort_flag, lim));
     if (ok) {
       tc_fence_after();
 #pragma unroll
@@ -970,7 +976,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsT<F8>, 1)
           l_own[g * HPG + h] = lt;
           st_async_f32(mapa(smem_u32(l_x + g * HPG + h), peer), lt, peer_bar);
         }
-        if (__all_sync(0xffffffffu, mbar_wait(bar(B::l_full), uc & 1, abort_flag))) {
+        if (__all_sync(0xffffffffu, mbar_wait(bar(B::l_full), uc & 1, abort_flag, lim))) {
           const float* m_fin = m_used + ((gt + n_tiles - 1) & 1) * NH + g * HPG;
           for (int h = lane; h < HPG; h += 32) {
             const int hg = g * HPG + h;
@@ -1058,22 +1064,37 @@ EncodeTiledFn encode_fn() {
 }
 
 // Unit counters of the persistent decode: one (claim, done) pair per launch in
-// flight, taken round robin from kCounterSlots per device.  A launch starts
-// with both at 0 and its last pair sets them back to 0, so consecutive
-// launches on a stream reuse a slot without a reset.  Launches that run
-// concurrently (different streams) take different slots; more than
-// kCounterSlots decode launches in flight at once on one device would share one.
+// flight, from kCounterSlots per device.  A launch starts with both at 0 and
+// its last pair sets them back to 0, so consecutive launches reuse a slot
+// without a reset.  The slot is chosen by the launch's o_part workspace: calls
+// that write the same o_part must not overlap on the GPU anyway (they would
+// race on the partials), and calls with different workspaces get different
+// slots while at most kCounterSlots distinct workspaces are in use.  A CUDA
+// graph captures the slot with the o_part it was captured with, so replays of
+// one graph share a slot exactly when they share a workspace.
 constexpr int kCounterSlots = 64;
+
 __device__ unsigned g_unit_claim[kCounterSlots];
 __device__ unsigned g_unit_done[kCounterSlots];
 
-bool claim_slot(unsigned** claim, unsigned** done) {
-  static std::atomic<unsigned> next{0};
+bool claim_slot(const void* workspace, unsigned** claim, unsigned** done) {
+  static std::mutex mu;
+  static const void* owner[kCounterSlots] = {};
+  static unsigned next = 0;
   void* c = nullptr;
   void* d = nullptr;
   if (cudaGetSymbolAddress(&c, g_unit_claim) != cudaSuccess || cudaGetSymbolAddress(&d, g_unit_done) != cudaSuccess)
     return false;
-  const unsigned i = next.fetch_add(1u) % kCounterSlots;
+  unsigned i = kCounterSlots;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    for (unsigned k = 0; k < (unsigned)kCounterSlots; ++k)
+      if (owner[k] == workspace) { i = k; break; }
+    if (i == (unsigned)kCounterSlots) {
+      i = next++ % kCounterSlots;
+      owner[i] = workspace;
+    }
+  }
   *claim = static_cast<unsigned*>(c) + i;
   *done = static_cast<unsigned*>(d) + i;
   return true;
@@ -1096,14 +1117,14 @@ cudaError_t launch_nh(const DecodeArgs& a, const CUtensorMap& tc, const CUtensor
   if (e != cudaSuccess) return e;
   TcParams p{a.n_heads, a.q_len, a.batch, a.block_table, a.max_pages, a.num_pages, a.seq_lens, a.num_splits,
              a.split_tokens, a.softmax_scale * 1.4426950408889634f, a.cache_scale, nullptr, nullptr,
-             a.o_part, a.lse_part, a.err};
+             a.o_part, a.lse_part, a.err, g_wait_limit.load(), g_withhold_q.load()};
   // Persistent pairs, one per SM pair, claiming units from a counter of this
   // launch: set-up, Q loads, pipeline fill and the epilogue are amortised and
   // overlapped across units, and splits of unequal length still balance.
   const long long units = (long long)a.batch * a.q_len * a.num_splits;
   const long long P = sm_pairs();
   const long long pairs = units < P ? units : P;
-  if (!claim_slot(&p.claim, &p.done)) return cudaErrorInvalidSymbol;
+  if (!claim_slot(a.o_part, &p.claim, &p.done)) return cudaErrorInvalidSymbol;
   dim3 grid((unsigned)(2 * pairs));
   decode_tc_kernel<NH, F8><<<grid, kThreadsT<F8>, LY::kSmem, st>>>(tc, tc2, tq, p);
   return cudaGetLastError();
@@ -1174,3 +1195,10 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st) {
 }
 
 }  // namespace mla
+
+extern "C" mla_status mla_test_set_decode_wait(unsigned long long limit_cycles, int withhold_q_load) {
+  if (limit_cycles == 0) limit_cycles = 4000000000ull;
+  mla::g_wait_limit.store(limit_cycles);
+  mla::g_withhold_q.store(withhold_q_load != 0);
+  return MLA_OK;
+}

@@ -165,6 +165,8 @@ mla_status mla_decode_fwd(const void* q_abs, mla_dtype q_dtype, const void* cach
   DecodeArgs a{q_abs, q_dtype, cache, cache_scale, cache_dtype, num_pages, block_table, max_pages_per_seq,
                page_size, seq_lens, batch, q_len, n_heads, num_splits, split_tokens, softmax_scale,
                o_part, lse_part, err_word};
+  if (decode_pair_supported(a))
+    return cuda_status(launch_decode_pair(a, stream), "mla_decode_fwd launch (tcgen05, head-split pairs)");
   if (decode_tc_supported(a)) return cuda_status(launch_decode_tc(a, stream), "mla_decode_fwd launch (tcgen05)");
   return cuda_status(launch_decode_simt(a, stream), "mla_decode_fwd launch");
 }

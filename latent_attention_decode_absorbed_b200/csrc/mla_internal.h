@@ -1,8 +1,11 @@
 // Internal declarations shared by the library's translation units.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+
+#include <atomic>
 
 #include "mla.h"
 
@@ -42,6 +45,9 @@ struct DecodeArgs {
   float* o_part; float* lse_part; int32_t* err;
 };
 cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t st);
+// tcgen05 path for 65..128 heads over a bf16 cache (heads split across a CTA pair)
+bool decode_pair_supported(const DecodeArgs& a);
+cudaError_t launch_decode_pair(const DecodeArgs& a, cudaStream_t st);
 // tcgen05 path: bf16 queries over a bf16 or e4m3 cache
 bool decode_tc_supported(const DecodeArgs& a);
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st);
@@ -51,5 +57,36 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st);
 cudaError_t launch_combine(const float* o_part, const float* lse_part, int rows, int n_heads,
                            int num_parts, bool shard_major, void* o_lat, int o_dtype, float* lse_out,
                            cudaStream_t st);
+
+// Bound (SM cycles, about 2 s at 2 GHz) of every barrier wait in the
+// tensor-core decode kernels, and the test hook that withholds one query load
+// (both set through mla_test_set_decode_wait, read at launch).
+inline std::atomic<unsigned long long> g_wait_limit{4000000000ull};
+inline std::atomic<int> g_withhold_q{0};
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
+typedef CUresult (*TensorMapEncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                      const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                      CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+inline TensorMapEncodeFn tensor_map_encoder() {
+  static TensorMapEncodeFn fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      return reinterpret_cast<TensorMapEncodeFn>(f);
+    return static_cast<TensorMapEncodeFn>(nullptr);
+  }();
+  return fn;
+}
+
+// CTA pairs that fit on the current device at one pair per two SMs.
+inline long long sm_pair_count() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 2)
+    return 1;
+  return sms / 2;
+}
 
 }  // namespace mla

@@ -214,6 +214,40 @@ __device__ __forceinline__ void mma_pair_f16(uint32_t d_tmem, uint64_t a_desc, u
       : "memory");
 }
 
+// The same, issued by a converged warp: one elected lane issues, the operands
+// are warp-uniform.
+__device__ __forceinline__ void mma_pair_f16_w(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                               uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// D[tmem] (+)= A[tmem] * B[smem]^T over one K=16 step for the pair, issued
+// by a converged warp (A from tensor memory: for M = 128 each CTA's 64 A rows
+// sit in lanes 0-63 of its own TMEM, 16 bf16 of K in 8 columns).
+__device__ __forceinline__ void mma_pair_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                              uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit_pair_w(uint32_t bar, uint16_t mask) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;\n\t}" ::"r"(bar),
+      "h"(mask)
+      : "memory");
+}
+
 // Arrive (once) on the barrier at the same offset in every CTA of `mask`
 // when all previously issued tcgen05 operations of this thread complete.
 __device__ __forceinline__ void mma_commit_pair(uint32_t bar, uint16_t mask) {

@@ -1,5 +1,5 @@
 """The C ABI without a GPU: libmla.so loads, exports every function that
-include/mla.h declares with the signature the binding uses, validates
+the headers in include/ declare with the signature the binding uses, validates
 arguments on the host, and its host-only RoPE table is right."""
 import ctypes
 import math
@@ -12,7 +12,8 @@ import pytest
 import latent_attention_decode_absorbed_b200 as mla
 from latent_attention_decode_absorbed_b200 import build as mla_build
 
-HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "mla.h")
+INCLUDE = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+HEADERS = sorted(os.path.join(INCLUDE, f) for f in os.listdir(INCLUDE) if f.endswith(".h"))
 
 
 @pytest.fixture(scope="module")
@@ -22,7 +23,7 @@ def lib():
 
 
 def _declarations():
-    text = open(HEADER).read()
+    text = "\n".join(open(h).read() for h in HEADERS)
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     decls = {}
     for m in re.finditer(r"(?:^|\n)\s*([A-Za-z_][\w\s\*]*?)\b(mla_\w+)\s*\(([^;{]*?)\)\s*;", text):
@@ -35,6 +36,8 @@ def _declarations():
 def _code(param: str) -> str:
     if "*" in param or param.startswith("cudaStream_t"):
         return "p"
+    if param.startswith("unsigned long long"):
+        return "Q"
     t = param.split()[0] if not param.startswith("const") else param.split()[1]
     return {"int": "i", "mla_dtype": "i", "float": "f", "double": "d"}[t]
 

@@ -206,6 +206,11 @@ CASES = [
     ("heads64_mtp_bf16", "bf16", [260], 2, 64, 128),
     ("heads48_bf16", "bf16", [200, 513], 1, 48, 256),
     ("long_split_bf16", "bf16", [5000], 1, 128, 4096),
+    # head counts that pad the pair's second half, and more units than CTA pairs
+    ("heads96_bf16", "bf16", [500, 90], 1, 96, 256),
+    ("heads80_mtp_bf16", "bf16", [300], 2, 80, 128),
+    ("heads65_bf16", "bf16", [129], 1, 65, 64),
+    ("many_units_bf16", "bf16", [1500] * 6 + [7000], 1, 128, 128),
     ("ragged_e4m3", "e4m3", [5, 400, 1025], 2, 128, 256),
     ("heads64_e4m3", "e4m3", [300, 70], 1, 64, 128),
     ("heads16_many_splits_e4m3", "e4m3", [700], 1, 16, 64),
