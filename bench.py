@@ -21,7 +21,6 @@ import hashlib
 import json
 import math
 import os
-import re
 import statistics
 import subprocess
 import sys
@@ -38,7 +37,7 @@ METRIC = "MLA decode tokens/s, latent-cache HBM GB/s and % of B200 roofline"
 CACHE_BYTES = {"f32": 2304, "bf16": 1152, "e4m3": 580}   # per cached row: 576 numbers (+ fp32 scale)
 DECODE_SRC = ["latent_attention_decode_absorbed_b200/csrc/decode_tc.cu",
               "latent_attention_decode_absorbed_b200/csrc/sm100.cuh"]
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_traffic.md")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_traffic.json")
 
 
 def peaks():
@@ -76,15 +75,14 @@ def decode_src_hash():
 
 
 def recorded_traffic(workload):
-    """DRAM bytes per decode launch from the committed ncu summary, if it was
-    taken on the current decode kernel source for this workload."""
+    """DRAM bytes per decode launch measured by ncu (profiles/decode_traffic.json),
+    if the entry was taken on the current decode kernel source for this workload."""
     if not os.path.exists(TRAFFIC_FILE):
         return None
     src = decode_src_hash()
-    for line in open(TRAFFIC_FILE):
-        m = re.match(r"\s*-?\s*traffic_per_launch\s+workload=(\S+)\s+src=(\S+)\s+bytes=(\d+)", line)
-        if m and m.group(1) == workload and m.group(2) == src:
-            return int(m.group(3))
+    for e in json.load(open(TRAFFIC_FILE)).get("entries", []):
+        if e.get("workload") == workload and e.get("src") == src:
+            return int(e["bytes"])
     return None
 
 
@@ -255,6 +253,42 @@ def workload_config(w, lens):
 
 
 # ------------------------------------------------------------------ GPU arm
+def _timed_steps(torch, step_fn, steps, stream, flush, barrier, decode_events=True):
+    """Time `steps` calls of step_fn(ev) on the device.  Without an L2 flush
+    the steps run back to back between two events; with one, the flush runs
+    before each step, outside that step's own pair of events, and the step
+    time is the sum of the per-step intervals.  Returns (total ms of the
+    timed steps, per-step decode-launch ms list)."""
+    dec = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) if decode_events else None
+           for _ in range(steps)]
+    barrier(); torch.cuda.synchronize()
+    if flush is None:
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for i in range(steps):
+            step_fn(dec[i])
+        t1.record(stream)
+        torch.cuda.synchronize(); barrier()
+        total = t0.elapsed_time(t1)
+    else:
+        se = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for i in range(steps):
+            flush.fill_(1.0)
+            se[i][0].record(stream)
+            step_fn(dec[i])
+            se[i][1].record(stream)
+        torch.cuda.synchronize(); barrier()
+        total = sum(a.elapsed_time(b) for a, b in se)
+    return total, [e[0].elapsed_time(e[1]) for e in dec] if decode_events else []
+
+
+def _decode_summary(alg_bytes, alg_flops, dec_ms, step_ms, pk):
+    roof_ms = 1e3 * max(alg_bytes / (pk["hbm_gbs"] * 1e9), alg_flops / (pk["bf16_tflops"] * 1e12))
+    return {"cache_gbs": alg_bytes / (dec_ms / 1e3) / 1e9, "tflops": alg_flops / (dec_ms / 1e3) / 1e12,
+            "tensor_frac_burst": alg_flops / (dec_ms / 1e3) / 1e12 / pk["bf16_tflops"],
+            "roofline_ms": roof_ms, "roofline_frac": roof_ms / dec_ms, "share_of_step": dec_ms / step_ms}
+
+
 def run_gpu(args, w, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -266,6 +300,8 @@ def run_gpu(args, w, rank, world, local_rank):
     lens = dw.lens
     stream = torch.cuda.current_stream(dev)
     alg_bytes, alg_flops = algorithmic(w, lens)
+    # workloads whose cache would stay in L2 get a 256 MB write before every
+    # step, outside the step's timed interval
     flush = None
     if alg_bytes <= 256e6:
         flush = torch.empty(int(256e6) // 4, dtype=torch.float32, device=dev)
@@ -275,8 +311,95 @@ def run_gpu(args, w, rank, world, local_rank):
             dist.barrier()
 
     def one_step(ev=None):
+        step.append(dw.kv_new, dw.seq_ids, dw.positions)
+        step.absorb(dw.q_nope, dw.q_pe, dw.w_uk)
+        if ev is not None:
+            ev[0].record(stream)
+        step.attend()
+        if ev is not None:
+            ev[1].record(stream)
+        step.combine()
+        step.project_out(dw.w_uv)
+
+    for _ in range(args.warmup):
         if flush is not None:
             flush.fill_(1.0)
+        one_step()
+    torch.cuda.synchronize()
+    assert int(step.err.item()) == 0, "device error flag set"
+    with ClockSampler(gpu_smi_id(local_rank)) as clk:
+        elapsed_ms, decode_ms = _timed_steps(torch, one_step, args.steps, stream, flush, barrier)
+    clocks = clk.summary()
+    # end-to-end through the public API: pinned host inputs in, host output back, every step
+    h_kv = dw.kv_new.cpu().pin_memory()
+    h_qn, h_qp = dw.q_nope.cpu().pin_memory(), dw.q_pe.cpu().pin_memory()
+    h_out = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
+    h2d = h_kv.numel() * h_kv.element_size() + h_qn.numel() * h_qn.element_size() + h_qp.numel() * h_qp.element_size()
+    d2h = h_out.numel() * h_out.element_size()
+
+    def e2e_step(ev=None):
+        dw.kv_new.copy_(h_kv, non_blocking=True)
+        dw.q_nope.copy_(h_qn, non_blocking=True)
+        dw.q_pe.copy_(h_qp, non_blocking=True)
+        step.run(dw.kv_new, dw.seq_ids, dw.positions, dw.q_nope, dw.q_pe, dw.w_uk, dw.w_uv)
+        h_out.copy_(step.out, non_blocking=True)
+
+    for _ in range(max(3, args.warmup)):
+        if flush is not None:
+            flush.fill_(1.0)
+        e2e_step()
+    e2e_ms, _ = _timed_steps(torch, e2e_step, args.steps, stream, flush, barrier, decode_events=False)
+    assert int(step.err.item()) == 0, "device error flag set"
+
+    # max over ranks
+    elapsed_ms, e2e_ms, dec_ms = max_over_ranks([elapsed_ms, e2e_ms, float(np.mean(decode_ms))], world, dev)
+    extra = None
+    if world == 1 and not args.no_extra and w.name == "long":
+        extra = time_extra(args, "fp8_mtp", dev, stream)
+    if rank != 0:
+        return 0
+    tokens_per_step = w.batch * w.q_len
+    value = job_throughput(world, tokens_per_step, args.steps, elapsed_ms)
+    e2e_value = job_throughput(world, tokens_per_step, args.steps, e2e_ms)
+    pk = peaks()
+    traffic = recorded_traffic(w.name)
+    roofline = binding_roofline(alg_bytes, alg_flops, dec_ms, pk, traffic)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
+        "data": "synthetic", "config": workload_config(w, lens),
+        "roofline": roofline,
+        "decode": _decode_summary(alg_bytes, alg_flops, dec_ms, elapsed_ms / args.steps, pk),
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": step.LAUNCHES_PER_STEP * args.steps,
+        "clocks": clocks,
+    }
+    if extra is not None:
+        line["fp8_mtp"] = extra
+    if not args.no_cpu_baseline and world == 1:
+        v, reps, el, cores = time_oracle(w, heads=w.n_heads, budget_s=args.cpu_budget)
+        line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                "sample": f"{reps} x sequence 0's {w.q_len} query row(s), all {w.n_heads} heads, "
+                                          f"over {int(lens[0])} cached rows ({el:.1f} s); absorbed fp64 oracle, "
+                                          f"cache built before timing"}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def time_extra(args, name, dev, stream):
+    """The same step on a second workload in the same process (the e4m3
+    two-token workload next to the long one): its decode launch against its
+    binding roofline, which for that workload is the tensor pipe."""
+    import torch
+    from workloads.device import DeviceWorkload
+    w = W.WORKLOADS[name]
+    dw = DeviceWorkload(w, device=dev)
+    step = dw.step
+    alg_bytes, alg_flops = algorithmic(w, dw.lens)
+    flush = torch.empty(int(256e6) // 4, dtype=torch.float32, device=dev) if alg_bytes <= 256e6 else None
+
+    def one_step(ev=None):
         step.append(dw.kv_new, dw.seq_ids, dw.positions)
         step.absorb(dw.q_nope, dw.q_pe, dw.w_uk)
         if ev is not None:
@@ -291,81 +414,19 @@ def run_gpu(args, w, rank, world, local_rank):
         one_step()
     torch.cuda.synchronize()
     assert int(step.err.item()) == 0, "device error flag set"
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(gpu_smi_id(local_rank)) as clk:
-        barrier(); torch.cuda.synchronize()
-        t_start.record(stream)
-        for i in range(args.steps):
-            one_step(evs[i])
-        t_end.record(stream)
-        torch.cuda.synchronize(); barrier()
-    elapsed_ms = t_start.elapsed_time(t_end)
-    decode_ms = [a.elapsed_time(b) for a, b in evs]
-    clocks = clk.summary()
-    # end-to-end through the public API: pinned host inputs in, host output back, every step
-    h_kv = dw.kv_new.cpu().pin_memory()
-    h_qn, h_qp = dw.q_nope.cpu().pin_memory(), dw.q_pe.cpu().pin_memory()
-    h_out = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
-    h2d = h_kv.numel() * h_kv.element_size() + h_qn.numel() * h_qn.element_size() + h_qp.numel() * h_qp.element_size()
-    d2h = h_out.numel() * h_out.element_size()
-
-    def e2e_step():
-        if flush is not None:
-            flush.fill_(1.0)
-        dw.kv_new.copy_(h_kv, non_blocking=True)
-        dw.q_nope.copy_(h_qn, non_blocking=True)
-        dw.q_pe.copy_(h_qp, non_blocking=True)
-        step.run(dw.kv_new, dw.seq_ids, dw.positions, dw.q_nope, dw.q_pe, dw.w_uk, dw.w_uv)
-        h_out.copy_(step.out, non_blocking=True)
-
-    for _ in range(max(3, args.warmup)):
-        e2e_step()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(); torch.cuda.synchronize()
-    e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize(); barrier()
-    e2e_ms = e0.elapsed_time(e1)
-    assert int(step.err.item()) == 0, "device error flag set"
-
-    # max over ranks
-    elapsed_ms, e2e_ms, dec_ms = max_over_ranks([elapsed_ms, e2e_ms, float(np.mean(decode_ms))], world, dev)
-    if rank != 0:
-        return 0
-    tokens_per_step = w.batch * w.q_len
-    value = job_throughput(world, tokens_per_step, args.steps, elapsed_ms)
-    e2e_value = job_throughput(world, tokens_per_step, args.steps, e2e_ms)
+    with ClockSampler(gpu_smi_id(dev.index or 0)) as clk:
+        total_ms, dec = _timed_steps(torch, one_step, args.steps, stream, flush, lambda: None)
     pk = peaks()
-    achieved = alg_bytes / (dec_ms / 1e3) / 1e9
-    traffic = recorded_traffic(w.name)
-    roofline = binding_roofline(alg_bytes, alg_flops, dec_ms, pk, traffic)
-    line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
-        "data": "synthetic", "config": workload_config(w, lens),
-        "roofline": roofline,
-        "decode": {"cache_gbs": achieved, "tflops": alg_flops / (dec_ms / 1e3) / 1e12,
-                   "tensor_frac_burst": alg_flops / (dec_ms / 1e3) / 1e12 / pk["bf16_tflops"],
-                   "roofline_ms": 1e3 * max(alg_bytes / (pk["hbm_gbs"] * 1e9), alg_flops / (pk["bf16_tflops"] * 1e12)),
-                   "roofline_frac": 1e3 * max(alg_bytes / (pk["hbm_gbs"] * 1e9),
-                                              alg_flops / (pk["bf16_tflops"] * 1e12)) / dec_ms,
-                   "share_of_step": dec_ms / (elapsed_ms / args.steps)},
-        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": step.LAUNCHES_PER_STEP * args.steps,
-        "clocks": clocks,
-    }
-    if not args.no_cpu_baseline and world == 1:
-        v, reps, el, cores = time_oracle(w, heads=w.n_heads, budget_s=args.cpu_budget)
-        line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                                "sample": f"{reps} x sequence 0's {w.q_len} query row(s), all {w.n_heads} heads, "
-                                          f"over {int(lens[0])} cached rows ({el:.1f} s); absorbed fp64 oracle, "
-                                          f"cache built before timing"}
-    print(json.dumps(line), flush=True)
-    return 0
+    dec_ms = float(np.mean(dec))
+    out = {"config": workload_config(w, dw.lens), "steps": args.steps,
+           "value": w.batch * w.q_len * args.steps / (total_ms / 1e3), "unit": "tokens/s",
+           "ms_per_step": total_ms / args.steps,
+           "roofline": binding_roofline(alg_bytes, alg_flops, dec_ms, pk, recorded_traffic(name)),
+           "decode": _decode_summary(alg_bytes, alg_flops, dec_ms, total_ms / args.steps, pk),
+           "clocks": clk.summary()}
+    del dw, step
+    torch.cuda.empty_cache()
+    return out
 
 
 def main():
@@ -377,6 +438,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="skip the e4m3 two-token line (long workload only)")
     # smaller cases of a workload's shape, for profiler captures (not bench lines)
     ap.add_argument("--batch", type=int, default=None, help="override the workload's batch (profiling)")
     ap.add_argument("--seq-len", type=int, default=None, help="override the workload's fixed length (profiling)")
