@@ -35,7 +35,8 @@ import workloads as W  # noqa: E402
 
 METRIC = "MLA decode tokens/s, latent-cache HBM GB/s and % of B200 roofline"
 CACHE_BYTES = {"f32": 2304, "bf16": 1152, "e4m3": 580}   # per cached row: 576 numbers (+ fp32 scale)
-DECODE_SRC = ["latent_attention_decode_absorbed_b200/csrc/decode_tc.cu",
+DECODE_SRC = ["latent_attention_decode_absorbed_b200/csrc/decode_pair.cu",
+              "latent_attention_decode_absorbed_b200/csrc/decode_tc.cu",
               "latent_attention_decode_absorbed_b200/csrc/sm100.cuh"]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_traffic.json")
 

@@ -29,6 +29,9 @@
  *   (mla_combine_shards: the same merge over the per-GPU results of sequences
  *    whose cached rows are sharded across GPUs)
  *   mla_out_uv        o_lat         -> out = W_UV o_lat                 (128 per head)
+ * and the projections on either side of that core:
+ *   mla_kv_proj_append  hidden states h -> kv_a = W_kv,a h -> cache rows (one kernel)
+ *   mla_out_proj        out (all heads) -> u = W_O [o_1; ...; o_H]
  *
  * Conventions for every entry point
  *  - Pointers named as device pointers must be device memory (or managed
@@ -182,8 +185,14 @@ mla_status mla_absorb_q(const void* q_nope, const void* q_pe, const void* w_uk, 
  *   o_part[r,h,s,:] = sum_j e^{z_j - m} c_j / sum_j e^{z_j - m}   over the split's visible j
  *   lse_part[r,h,s] = m + ln sum_j e^{z_j - m}  (natural log)
  *   A split with no visible row gets lse_part = -inf; its o_part is left
- *   unwritten by the tensor-core path (zero on the fp32 path), and
+ *   unwritten by the tensor-core paths (zero on the fp32 path), and
  *   mla_combine gives it weight 0 without reading it.
+ *   The tensor-core path for more than 64 heads over a bf16 cache may work a
+ *   run of consecutive splits of one query row as one unit (it does so when
+ *   there are at least four splits per CTA pair of the GPU): it then writes
+ *   the run's merged partial (the same formulas over the run's rows) at the
+ *   run's first split and lse_part = -inf at its other splits, whose o_part
+ *   stays unwritten.  mla_combine returns the same result either way.
  *   q_abs       device [batch*q_len, n_heads, 576], q_dtype F32 or BF16
  *   cache       device [num_pages, 9, 64, 64], page-blocked; cache_scale as for mla_cache_append
  *   block_table device int32 [batch, max_pages_per_seq]
@@ -270,6 +279,54 @@ mla_status mla_combine_shards(const float* o_shard, const float* lse_shard, int 
  */
 mla_status mla_out_uv(const void* o_lat, const void* w_uv, void* out, int rows, int n_heads,
                       mla_dtype dtype, cudaStream_t stream);
+
+/*
+ * mla_out_proj
+ * Output projection after the value up-projection ("DeepSeek-V2: MLA
+ * Explained", "MLA Full Formulas" part 3: u_t = W_O [o_{t,1}; ...; o_{t,n_h}],
+ * the heads concatenated in head order):
+ *   u[r, j] = sum_{h, i} W_O[j, h*128 + i] * out[r, h, i]     (fp32 accumulate)
+ *   out  device bf16 [rows, n_heads, 128]   (mla_out_uv's result; at decode
+ *        row counts it is still in L2 when this call reads it)
+ *   w_o  device bf16 [d_model, n_heads*128]
+ *   u    device float [rows, d_model], overwritten
+ *   d_model a multiple of 256.  Runs on the tcgen05 tensor cores as a split-K
+ *   GEMM whose fp32 partial tiles are added into u (so bits may differ
+ *   between runs in the last place); u is cleared first on the same stream.
+ */
+mla_status mla_out_proj(const void* out, const void* w_o, float* u, int rows, int n_heads, int d_model,
+                        cudaStream_t stream);
+
+/*
+ * mla_kv_proj_workspace_bytes (host function, no GPU needed)
+ * Bytes of caller workspace mla_kv_proj_append needs: the fp32 kv_a rows
+ * [n_new, 576] plus one counter per 128 tokens.  0 for n_new <= 0.
+ */
+size_t mla_kv_proj_workspace_bytes(int n_new);
+
+/*
+ * mla_kv_proj_append
+ * The joint KV down-projection and the cache append in one kernel ("KV
+ * Compression - DeepSeek-V3", "How it works", Eq. (1):
+ * [c_t^KV ; k~_t^R] = W_kv,a h_t, 576 wide, then split [512, 64], RMSNorm the
+ * latent, RoPE the rope part, store; "Official code": wkv_a, kv_norm):
+ *   kv_a[n, :] = sum_k W_kv,a[:, k] * h[n, k]                (fp32 accumulate)
+ *   then exactly mla_cache_append's row writer on the fp32 kv_a rows.
+ *   h       device bf16 [n_new, d_model];  w_kva device bf16 [576, d_model]
+ *   d_model a multiple of 64
+ *   workspace device, mla_kv_proj_workspace_bytes(n_new) bytes, 16-byte
+ *           aligned, caller-owned; cleared by the call (on the stream); on
+ *           completion its first n_new*576 floats hold the fp32 kv_a rows
+ *   the other arguments as for mla_cache_append
+ * A split-K GEMM on the tcgen05 tensor cores reduces into the workspace; the
+ * last CTA to finish a tile of 128 tokens writes those tokens' cache rows.
+ */
+mla_status mla_kv_proj_append(const void* h, const void* w_kva, int n_new, int d_model, void* workspace,
+                              const int32_t* seq_ids, const int32_t* positions, const int32_t* block_table,
+                              int batch, int max_pages_per_seq, int page_size, const float* norm_gain, float eps,
+                              const float* rope_cos, const float* rope_sin, int rope_max_pos, void* cache,
+                              float* cache_scale, mla_dtype cache_dtype, int num_pages, int32_t* err_word,
+                              cudaStream_t stream);
 
 /*
  * mla_decode_static

@@ -35,6 +35,9 @@ _SIGS = {
     "mla_out_uv": ("i", "pppiiip"),
     "mla_decode_static": ("i", "pippiipiipiiiiifpippp"),
     "mla_test_set_decode_wait": ("i", "Qi"),
+    "mla_out_proj": ("i", "pppiiip"),
+    "mla_kv_proj_workspace_bytes": ("z", "i"),
+    "mla_kv_proj_append": ("i", "ppiippppiiipfppippiipp"),
 }
 _CT = {"p": ctypes.c_void_p, "i": ctypes.c_int, "f": ctypes.c_float, "d": ctypes.c_double,
        "s": ctypes.c_char_p, "z": ctypes.c_size_t, "Q": ctypes.c_ulonglong}
@@ -182,6 +185,27 @@ def mla_decode_static(q_abs, q_dtype, cache, cache_scale, cache_dtype, num_pages
 
 
 MLA_STATIC_MAX_PARTIALS = 8192
+
+
+def mla_out_proj(out, w_o, u, rows, n_heads, d_model, stream=None):
+    """u[r] = W_O [out[r, 0]; ...; out[r, H-1]] (fp32 u, overwritten)."""
+    _check("mla_out_proj", lib().mla_out_proj(_ptr(out), _ptr(w_o), _ptr(u), int(rows), int(n_heads), int(d_model),
+                                              _stream(stream)))
+
+
+def mla_kv_proj_workspace_bytes(n_new) -> int:
+    return int(lib().mla_kv_proj_workspace_bytes(int(n_new)))
+
+
+def mla_kv_proj_append(h, w_kva, n_new, d_model, workspace, seq_ids, positions, block_table, batch,
+                       max_pages_per_seq, page_size, norm_gain, eps, rope_cos, rope_sin, rope_max_pos, cache,
+                       cache_scale, cache_dtype, num_pages, err_word=None, stream=None):
+    """kv_a = W_kv,a h, then mla_cache_append's row writer, in one kernel."""
+    _check("mla_kv_proj_append", lib().mla_kv_proj_append(
+        _ptr(h), _ptr(w_kva), int(n_new), int(d_model), _ptr(workspace), _ptr(seq_ids), _ptr(positions),
+        _ptr(block_table), int(batch), int(max_pages_per_seq), int(page_size), _ptr(norm_gain), float(eps),
+        _ptr(rope_cos), _ptr(rope_sin), int(rope_max_pos), _ptr(cache), _ptr(cache_scale), int(cache_dtype),
+        int(num_pages), _ptr(err_word), _stream(stream)))
 
 
 def mla_test_set_decode_wait(limit_cycles=0, withhold_q_load=False):

@@ -78,8 +78,8 @@ constexpr int kOffMisc = kOffP + 4 * kPChunk;
 constexpr int kMBars = 0;                 // 48 barriers
 constexpr int kMTmem = 48 * 8;
 constexpr int kMAbort = kMTmem + 4;
-constexpr int kMRedMax = kMTmem + 16;     // float [2 lane halves][2 column halves][64 heads]
-constexpr int kMRedSum = kMRedMax + 4 * kHPC * 4;
+constexpr int kMRedMax = kMTmem + 16;     // float [2 tile parities][2 lane halves][2 column halves][64 heads]
+constexpr int kMRedSum = kMRedMax + 2 * 4 * kHPC * 4;   // float [2 lane halves][2 column halves][64 heads]
 constexpr int kMUnitQ = kMRedSum + 4 * kHPC * 4;
 constexpr int kMiscBytes = kMUnitQ + 4 * kQN;
 constexpr int kSmem = kOffMisc + kMiscBytes + 1024;       // + alignment slack
@@ -106,6 +106,7 @@ struct PairParams {
   int max_pages, num_pages;
   const int32_t* seq_lens;
   int num_splits, split_tokens;
+  int run;                     // splits per claimed unit (consecutive in (query row, split) order)
   float scale_log2;            // softmax_scale * log2(e)
   unsigned* claim;             // unit counter of this launch (0 at launch; reset by the last pair)
   unsigned* done;              // pairs finished
@@ -159,21 +160,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t peer = rank ^ 1u;
   const bool leader = rank == 0;
 
-  // ---- units: (query row r, split s), claimed by persistent pairs; every
-  // role walks the pair's same sequence, so barrier phases count globally
+  // ---- units: runs of `run` consecutive splits in (query row, split) order,
+  // claimed by persistent pairs; a run that crosses into the next query row
+  // is worked as two segments.  Every role walks the pair's same sequence of
+  // segments, so barrier phases count globally (ring stages, tiles, segments).
+  // A segment's splits are merged in TMEM: its partial is written at its
+  // first split, and its other splits get lse = -inf (weight 0 in the merge).
   const int S = p.num_splits;
-  const int n_units = p.batch * p.q_len * S;
+  const int n_flat = p.batch * p.q_len * S;
+  const int n_units = (n_flat + p.run - 1) / p.run;
   const int n_pairs = gridDim.x >> 1;
-  struct UnitInfo { int r, s, b, lo, hi, n_tiles; };
-  auto unit_at = [&](int u) -> UnitInfo {
+  struct UnitInfo { int r, s, s1, b, lo, hi, n_tiles; };
+  // the segment starting at flat split f of a unit that ends at f1
+  auto seg_at = [&](int f, int f1) -> UnitInfo {
     UnitInfo x;
-    x.r = u / S;
-    x.s = u % S;
+    x.r = f / S;
+    x.s = f - x.r * S;
+    x.s1 = min(S, x.s + (f1 - f));
     x.b = x.r / p.q_len;
     const int t = x.r % p.q_len;
     const int n_vis = p.seq_lens[x.b] - p.q_len + t + 1;
     x.lo = x.s * p.split_tokens;
-    x.hi = min(x.lo + p.split_tokens, n_vis);
+    x.hi = (int)min((long long)x.s1 * p.split_tokens, (long long)n_vis);
     const int n_tok = x.hi - x.lo;
     x.n_tiles = n_tok > 0 ? (n_tok + kTile - 1) / kTile : 0;
     return x;
@@ -275,7 +283,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       if (u == -2) { ok = false; break; }
       if (u < 0) break;
-      const UnitInfo U = unit_at(u);
+      const int f1 = min(n_flat, (u + 1) * p.run);
+      for (int f = u * p.run; f < f1 && ok;) {
+      const UnitInfo U = seg_at(f, f1);
+      f += U.s1 - U.s;
       if (U.n_tiles == 0) continue;
       const int r = U.r, b = U.b, lo = U.lo, hi = U.hi, n_tiles = U.n_tiles;
       if (lane == 0) {
@@ -323,12 +334,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (ok) ok = load_o(i);
       }
       ++uc;
+      }
     }
   } else if (warp == kWarpMma) {
     // ================= MMA issuer (leader CTA, whole warp, one elected lane) =================
-    // Per unit: S(0), then per tile i: S(i+1), O(i).  S(i+1) goes to the
-    // other TMEM buffer while the softmax of tile i reads S(i); S(i+2) reuses
-    // S(i)'s columns after O(i), which waited for the softmax of tile i.
+    // Per unit: S(0), then per tile i: S(i+1), O(i).  S(i+1) goes to the other
+    // TMEM buffer while the softmax of tile i reads S(i); S(i+2) reuses S(i)'s
+    // columns after O(i), which waited for the softmax of tile i to finish
+    // (tcgen05.mma operations of one thread execute in issue order).  The
+    // value GEMM of tile i waits for P(i), which the softmax writes after
+    // O(i-1) is done (one P buffer), so running the score GEMM further ahead
+    // only delays O(i) (measured slower).
     if (leader) {
       constexpr uint32_t idS = idesc_f16(128, 256, false, false);
       constexpr uint32_t idO = idesc_f16(128, 256, false, true);
@@ -348,14 +364,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int u = next_unit(k);
         if (u == -2) { ok = false; break; }
         if (u < 0) break;
-        const UnitInfo U = unit_at(u);
+        const int f1 = min(n_flat, (u + 1) * p.run);
+        for (int f = u * p.run; f < f1 && ok;) {
+        const UnitInfo U = seg_at(f, f1);
+        f += U.s1 - U.s;
         if (U.n_tiles == 0) continue;
         const int lo = U.lo, hi = U.hi, n_tiles = U.n_tiles;
         ok = __all_sync(0xffffffffu, mbar_wait(bar(kBQFull), uc & 1, abort_flag, lim));
         if (!ok) break;
         tc_fence_after();
         auto issue_s = [&](int i) -> bool {
-          const uint32_t sb = (gt + i) & 1u;
+          const uint32_t t = gt + i;
+          const uint32_t sb = t & 1u;
           const uint32_t d = tmem + kColS + 128 * sb;
           const uint64_t qd = smem_desc_sw128(s_q, 16, 1024);
           for (int c = 0; c < kChunks; ++c) {
@@ -405,6 +425,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         gt += n_tiles;
         ++uc;
+        }
       }
     }
   } else {
@@ -435,11 +456,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int u = next_unit(k);
       if (u == -2) { ok = false; break; }
       if (u < 0) break;
-      const UnitInfo U = unit_at(u);
+      const int f1 = min(n_flat, (u + 1) * p.run);
+      for (int f = u * p.run; f < f1 && ok;) {
+      const UnitInfo U = seg_at(f, f1);
+      f += U.s1 - U.s;
       const int r = U.r, s = U.s, b = U.b, lo = U.lo, hi = U.hi, n_tiles = U.n_tiles;
+      // splits of the segment after its first: merged into the first (lse = -inf,
+      // o_part unwritten: the merge gives them weight 0 and does not read them)
+      if (part == 0 && head < p.n_heads)
+        for (int s2 = s + 1; s2 < U.s1; ++s2) p.lse_part[((size_t)r * p.n_heads + head) * S + s2] = -INFINITY;
       if (n_tiles == 0) {
-        // nothing visible in this split: lse = -inf; o_part is left unwritten
-        // (the merge gives such a split weight 0 and does not read it)
+        // nothing visible in the segment: lse = -inf at its first split too
         if (part == 0 && head < p.n_heads) p.lse_part[((size_t)r * p.n_heads + head) * S + s] = -INFINITY;
         continue;
       }
@@ -447,15 +474,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       for (int i = 0; i < n_tiles; ++i) {
         const uint32_t t = gt + i;
         const uint32_t sb = t & 1u;
-        ok = __all_sync(0xffffffffu, mbar_wait<false>(bar(kBSFull + sb), (t >> 1) & 1, abort_flag, lim));
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t scol = tmem + lane_addr + kColS + 128 * sb;
-        float v[64];
-        tmem_ld<32>(scol + 64 * ch, v);
-        tmem_ld<32>(scol + 64 * ch + 32, v + 32);
-        tmem_wait_ld();
-        // rows of this thread: one page of the sequence
+        // rows of this thread: one page of the sequence (its table entry is
+        // read before the wait for the scores, off the critical path)
         const int row0 = lo + kTile * i + 128 * half + 64 * ch;
         int nvalid = min(max(hi - row0, 0), 64);
         if (nvalid > 0) {
@@ -466,16 +486,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             flag_error(p.err, MLA_DEVERR_PAGE);
           }
         }
+        ok = __all_sync(0xffffffffu, mbar_wait<false>(bar(kBSFull + sb), (t >> 1) & 1, abort_flag, lim));
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t scol = tmem + lane_addr + kColS + 128 * sb;
+        float v[64];
+        tmem_ld<32>(scol + 64 * ch, v);
+        tmem_ld<32>(scol + 64 * ch + 32, v + 32);
+        tmem_wait_ld();
         float mx = -INFINITY;
 #pragma unroll
         for (int j = 0; j < 64; ++j) {
           v[j] = j < nvalid ? v[j] * p.scale_log2 : -INFINITY;
           mx = fmaxf(mx, v[j]);
         }
-        red_max[part * kHPC + hh] = mx;
+        // the four partial maxima of each head, double-buffered by tile parity:
+        // a warp writes the next tile's slot only after passing this tile's
+        // sync, so no warp can overwrite a slot that another is still reading
+        float* rm = red_max + sb * 4 * kHPC;
+        rm[part * kHPC + hh] = mx;
         if (!(ok = soft_sync(0))) break;
-        const float tmax = fmaxf(fmaxf(red_max[hh], red_max[kHPC + hh]),
-                                 fmaxf(red_max[2 * kHPC + hh], red_max[3 * kHPC + hh]));
+        const float tmax = fmaxf(fmaxf(rm[hh], rm[kHPC + hh]), fmaxf(rm[2 * kHPC + hh], rm[3 * kHPC + hh]));
         const float m_new = (tmax > m_run + kRescaleLog2) ? tmax : m_run;
         const bool changed = m_new != m_run;
         // factor for the sums and the accumulator kept so far (0 when nothing was kept)
@@ -563,6 +594,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       gt += n_tiles;
       ++uc;
+      }
     }
   }
 
@@ -658,12 +690,21 @@ cudaError_t launch_decode_pair(const DecodeArgs& a, cudaStream_t st) {
   }
   cudaError_t e = cudaFuncSetAttribute(decode_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (e != cudaSuccess) return e;
-  PairParams p{a.n_heads, a.q_len, a.batch, a.block_table, a.max_pages, a.num_pages, a.seq_lens, a.num_splits,
-               a.split_tokens, a.softmax_scale * 1.4426950408889634f, nullptr, nullptr, a.o_part, a.lse_part, a.err,
-               g_wait_limit.load(), g_withhold_q.load()};
-  if (!claim_slot(a.o_part, &p.claim, &p.done)) return cudaErrorInvalidSymbol;
-  const long long units = (long long)a.batch * a.q_len * a.num_splits;
+  // Runs of splits per claimed unit.  With at least four splits per CTA pair,
+  // every pair gets one run of ceil(splits / pairs) consecutive splits: each
+  // pair then writes one or two partials instead of one per split (the fp32
+  // partials were 11 % of the bytes of the long workload's launch, and each
+  // epilogue sits on the pair's critical path).  With fewer splits, as in
+  // batches of short ragged sequences, single splits keep the dynamic
+  // claiming balanced.
   const long long P = sm_pair_count();
+  const long long n_flat = (long long)a.batch * a.q_len * a.num_splits;
+  const int run = n_flat >= 4 * P ? (int)((n_flat + P - 1) / P) : 1;
+  const long long units = (n_flat + run - 1) / run;
+  PairParams p{a.n_heads, a.q_len, a.batch, a.block_table, a.max_pages, a.num_pages, a.seq_lens, a.num_splits,
+               a.split_tokens, run, a.softmax_scale * 1.4426950408889634f, nullptr, nullptr, a.o_part, a.lse_part,
+               a.err, g_wait_limit.load(), g_withhold_q.load()};
+  if (!claim_slot(a.o_part, &p.claim, &p.done)) return cudaErrorInvalidSymbol;
   const long long pairs = units < P ? units : P;
   decode_pair_kernel<<<dim3((unsigned)(2 * pairs)), kThreads, kSmem, st>>>(tc, tc2, tq, p);
   return cudaGetLastError();

@@ -171,6 +171,58 @@ mla_status mla_decode_fwd(const void* q_abs, mla_dtype q_dtype, const void* cach
   return cuda_status(launch_decode_simt(a, stream), "mla_decode_fwd launch");
 }
 
+mla_status mla_out_proj(const void* out, const void* w_o, float* u, int rows, int n_heads, int d_model,
+                        cudaStream_t stream) {
+  MLA_REQUIRE(rows >= 0, MLA_ERR_INVALID_ARG, "mla_out_proj: rows < 0");
+  MLA_REQUIRE(n_heads >= 1 && n_heads <= MLA_MAX_HEADS, MLA_ERR_INVALID_ARG, "mla_out_proj: n_heads must be in [1, %d]",
+              MLA_MAX_HEADS);
+  MLA_REQUIRE(d_model >= 256 && d_model % 256 == 0 && d_model <= 65536, MLA_ERR_UNSUPPORTED,
+              "mla_out_proj: d_model must be a multiple of 256 in [256, 65536]");
+  MLA_REQUIRE(rows <= 65535 * 128, MLA_ERR_UNSUPPORTED, "mla_out_proj: rows above %d", 65535 * 128);
+  if (rows == 0) return MLA_OK;
+  MLA_REQUIRE(out && w_o && u, MLA_ERR_INVALID_ARG, "mla_out_proj: null pointer");
+  MLA_REQUIRE(aligned(out, 16) && aligned(w_o, 16) && aligned(u, 16), MLA_ERR_INVALID_ARG,
+              "mla_out_proj: pointers must be 16-byte aligned");
+  return cuda_status(launch_out_proj(out, w_o, u, rows, n_heads, d_model, stream), "mla_out_proj launch");
+}
+
+size_t mla_kv_proj_workspace_bytes(int n_new) {
+  if (n_new <= 0) return 0;
+  return (size_t)n_new * MLA_D_ROW * sizeof(float) + (size_t)((n_new + 127) / 128) * sizeof(unsigned);
+}
+
+mla_status mla_kv_proj_append(const void* h, const void* w_kva, int n_new, int d_model, void* workspace,
+                              const int32_t* seq_ids, const int32_t* positions, const int32_t* block_table,
+                              int batch, int max_pages_per_seq, int page_size, const float* norm_gain, float eps,
+                              const float* rope_cos, const float* rope_sin, int rope_max_pos, void* cache,
+                              float* cache_scale, mla_dtype cache_dtype, int num_pages, int32_t* err_word,
+                              cudaStream_t stream) {
+  MLA_REQUIRE(n_new >= 0, MLA_ERR_INVALID_ARG, "mla_kv_proj_append: n_new < 0");
+  MLA_REQUIRE(d_model >= 64 && d_model % 64 == 0 && d_model <= 65536, MLA_ERR_UNSUPPORTED,
+              "mla_kv_proj_append: d_model must be a multiple of 64 in [64, 65536]");
+  MLA_REQUIRE(cache_dtype == MLA_F32 || cache_dtype == MLA_BF16 || cache_dtype == MLA_E4M3, MLA_ERR_UNSUPPORTED,
+              "mla_kv_proj_append: bad cache_dtype");
+  MLA_REQUIRE(page_size == MLA_PAGE, MLA_ERR_UNSUPPORTED, "mla_kv_proj_append: page_size must be %d", MLA_PAGE);
+  MLA_REQUIRE(batch >= 1 && max_pages_per_seq >= 1 && num_pages >= 1 && rope_max_pos >= 1, MLA_ERR_INVALID_ARG,
+              "mla_kv_proj_append: batch, max_pages_per_seq, num_pages, rope_max_pos must be >= 1");
+  MLA_REQUIRE(eps >= 0.f && isfinite(eps), MLA_ERR_INVALID_ARG, "mla_kv_proj_append: eps must be finite and >= 0");
+  MLA_REQUIRE((long long)max_pages_per_seq * page_size < (1ll << 31), MLA_ERR_INVALID_ARG,
+              "mla_kv_proj_append: table capacity overflows int32 positions");
+  MLA_REQUIRE(n_new <= 65535 * 128, MLA_ERR_UNSUPPORTED, "mla_kv_proj_append: n_new above %d", 65535 * 128);
+  if (n_new == 0) return MLA_OK;
+  MLA_REQUIRE(h && w_kva && workspace && seq_ids && positions && block_table && rope_cos && rope_sin && cache,
+              MLA_ERR_INVALID_ARG, "mla_kv_proj_append: null pointer");
+  MLA_REQUIRE(cache_dtype != MLA_E4M3 || cache_scale, MLA_ERR_INVALID_ARG,
+              "mla_kv_proj_append: E4M3 cache needs cache_scale");
+  MLA_REQUIRE(aligned(h, 16) && aligned(w_kva, 16) && aligned(workspace, 16) && aligned(cache, 16) &&
+                  aligned(norm_gain, 16),
+              MLA_ERR_INVALID_ARG, "mla_kv_proj_append: h, w_kva, workspace, cache and norm_gain must be 16-byte aligned");
+  AppendArgs a{nullptr, MLA_F32, n_new, seq_ids, positions, block_table, batch, max_pages_per_seq, page_size,
+               norm_gain, eps, rope_cos, rope_sin, rope_max_pos, cache, cache_scale, cache_dtype, num_pages, err_word};
+  return cuda_status(launch_kv_proj_append(h, w_kva, d_model, static_cast<float*>(workspace), a, stream),
+                     "mla_kv_proj_append launch");
+}
+
 mla_status mla_combine(const float* o_part, const float* lse_part, int rows, int n_heads, int num_splits,
                        void* o_lat, mla_dtype o_dtype, float* lse_out, cudaStream_t stream) {
   MLA_REQUIRE(rows >= 0 && n_heads >= 1 && n_heads <= MLA_MAX_HEADS && num_splits >= 1, MLA_ERR_INVALID_ARG,

@@ -52,6 +52,12 @@ cudaError_t launch_decode_pair(const DecodeArgs& a, cudaStream_t st);
 bool decode_tc_supported(const DecodeArgs& a);
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st);
 
+// split-K tcgen05 GEMMs of the projections around the attention core
+cudaError_t launch_out_proj(const void* out_heads, const void* w_o, float* u, int rows, int n_heads, int d_model,
+                            cudaStream_t st);
+cudaError_t launch_kv_proj_append(const void* h, const void* w_kva, int d_model, float* workspace,
+                                  const AppendArgs& a, cudaStream_t st);
+
 // shard_major: parts laid out [num_parts, rows, n_heads, 512] (per-GPU results
 // of a row-sharded sequence) instead of [rows, n_heads, num_parts, 512]
 cudaError_t launch_combine(const float* o_part, const float* lse_part, int rows, int n_heads,
