@@ -251,20 +251,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tm_cache2);
       tma_prefetch_desc(&tm_q);
     }
-    auto take = [&](uint32_t bytes, uint32_t& dst, uint32_t& fb) -> bool {
-      const uint32_t slot = kc % kSlots;
-      const uint32_t ph = (kc / kSlots) & 1u;
-      bool ok = true;
-      if (lane == 0) {
-        ok = mbar_wait<false>(bar(kBEmpty + slot), ph ^ 1u, abort_flag, lim);
-        if (ok && leader) mbar_arrive_expect_tx(bar(kBFull + slot), 2u * bytes);
-      }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      dst = s_ring + slot * kSlotBytes;
-      fb = mapa(bar(kBFull + slot), 0);
-      ++kc;
-      return ok;
-    };
     // score rows are re-read by the value stages of the pair (this CTA's for
     // its dims, the peer's for the other dims) one tile later: evict-last;
     // value loads are the rows' last use: evict-first
@@ -303,36 +289,74 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
-      auto load_s = [&](int i) -> bool {
-        bool vv;
-        const int pg = page_of(p, b, lo + kTile * i + 128 * (int)rank + 64 * (lane & 1), &vv);
-        for (int c = 0; c < kChunks; ++c) {
-          uint32_t dst, fb;
-          if (!take(kSlotBytes, dst, fb)) return false;
-          if (lane < 2) tma_load_2d_pair_hint(dst + lane * kBox, &tm_cache, 0, (pg * kChunks + c) * 64, fb, pol_keep);
-        }
-        return true;
-      };
-      auto load_o = [&](int j) -> bool {
-        for (int pg_i = 0; pg_i < 4; ++pg_i) {
-          const int row0 = lo + kTile * j + 64 * pg_i;
-          if (row0 >= hi) break;
-          bool vld;
-          const int pg = page_of(p, b, row0, &vld);
-          for (int bb = 0; bb < 2; ++bb) {
+      // One lane issues every copy of the segment: a per-stage hand-off
+      // between lanes (shuffles, a converged wait) cost ~4 % of the launch.
+      // The table entries of tile i + 2 are fetched while tile i is issued,
+      // so their latency stays off the stream.
+      if (lane == 0) {
+        const int32_t* bt = p.block_table + (size_t)b * p.max_pages;
+        const int pb = lo >> 6;      // the segment's first page index (lo is a multiple of 64)
+        auto entry = [&](int pidx) -> int { return pidx < p.max_pages ? __ldg(bt + pidx) : -1; };
+        // rows outside the table or the pool read page 0 (readable; they are masked)
+        auto page = [&](int pg) -> int { return pg >= 0 && pg < p.num_pages ? pg : 0; };
+        auto take = [&](uint32_t& dst, uint32_t& fb) -> bool {
+          const uint32_t slot = kc % kSlots;
+          const uint32_t ph = (kc / kSlots) & 1u;
+          if (!mbar_wait<false>(bar(kBEmpty + slot), ph ^ 1u, abort_flag, lim)) return false;
+          if (leader) mbar_arrive_expect_tx(bar(kBFull + slot), 2u * kSlotBytes);
+          dst = s_ring + slot * kSlotBytes;
+          fb = mapa(bar(kBFull + slot), 0);
+          ++kc;
+          return true;
+        };
+        // score stages: column chunk c of this CTA's two pages of the tile
+        auto load_s = [&](int pg0, int pg1) -> bool {
+          for (int c = 0; c < kChunks; ++c) {
             uint32_t dst, fb;
-            if (!take(kSlotBytes, dst, fb)) return false;
-            if (lane == 0)
-              tma_load_2d_pair_hint(dst, &tm_cache2, 0, (pg * kChunks + 4 * bb + 2 * (int)rank) * 64, fb, pol_drop);
+            if (!take(dst, fb)) return false;
+            tma_load_2d_pair_hint(dst, &tm_cache, 0, (pg0 * kChunks + c) * 64, fb, pol_keep);
+            tma_load_2d_pair_hint(dst + kBox, &tm_cache, 0, (pg1 * kChunks + c) * 64, fb, pol_keep);
+          }
+          return true;
+        };
+        // value stages: per page of tile j with visible rows, this CTA's two dims blocks pairs
+        auto load_o = [&](int j, const int (&pg)[4]) -> bool {
+#pragma unroll
+          for (int pg_i = 0; pg_i < 4; ++pg_i) {
+            if (lo + kTile * j + 64 * pg_i >= hi) break;
+            for (int bb = 0; bb < 2; ++bb) {
+              uint32_t dst, fb;
+              if (!take(dst, fb)) return false;
+              tma_load_2d_pair_hint(dst, &tm_cache2, 0, (pg[pg_i] * kChunks + 4 * bb + 2 * (int)rank) * 64, fb,
+                                    pol_drop);
+            }
+          }
+          return true;
+        };
+        int cur[4], nxt[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          cur[q] = entry(pb + q);
+          nxt[q] = entry(pb + 4 + q);
+        }
+        ok = load_s(page(rank ? cur[2] : cur[0]), page(rank ? cur[3] : cur[1]));
+        for (int i = 0; i < n_tiles && ok; ++i) {
+          int ahead[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) ahead[q] = entry(pb + 4 * (i + 2) + q);
+          if (i + 1 < n_tiles) ok = load_s(page(rank ? nxt[2] : nxt[0]), page(rank ? nxt[3] : nxt[1]));
+          int pg[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) pg[q] = page(cur[q]);
+          if (ok) ok = load_o(i, pg);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            cur[q] = nxt[q];
+            nxt[q] = ahead[q];
           }
         }
-        return true;
-      };
-      ok = load_s(0);
-      for (int i = 0; i < n_tiles && ok; ++i) {
-        if (i + 1 < n_tiles) ok = load_s(i + 1);
-        if (ok) ok = load_o(i);
       }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
       ++uc;
       }
     }
