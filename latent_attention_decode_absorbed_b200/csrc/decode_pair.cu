@@ -188,6 +188,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   };
 
   // ---- set-up
+  // the pair's first unit is claimed now, so that the counter's round trip
+  // overlaps the barrier and tensor-memory set-up
+  unsigned first_claim = 0;
+  if (leader && threadIdx.x == 0) first_claim = atomicAdd(p.claim, 1u);
   if (threadIdx.x == 0) {
     for (int i = 0; i < kSlots; ++i) {
       mbar_init(bar(kBFull + i), 1);
@@ -220,7 +224,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   auto claim = [&](uint32_t k) -> int {      // leader producer, lane 0
     const uint32_t slot = k % kQN;
     if (k >= kQN && !mbar_wait(bar(kBUqEmpty + slot), ((k / kQN) - 1) & 1, abort_flag, lim)) return -2;
-    const unsigned cu = atomicAdd(p.claim, 1u);
+    const unsigned cu = k == 0 ? first_claim : atomicAdd(p.claim, 1u);
     const int uu = cu < (unsigned)n_units ? (int)cu : -1;
     *reinterpret_cast<volatile int*>(unit_q + slot) = uu;
     st_cluster_b32(mapa(smem_u32(unit_q + slot), peer), (uint32_t)uu);
@@ -592,24 +596,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (ok) {
         const float lt = red_sum[hh] + red_sum[kHPC + hh] + red_sum[2 * kHPC + hh] + red_sum[3 * kHPC + hh];
         const float inv_l = lt > 0.f ? 1.0f / lt : 0.f;
-        const bool live = head < p.n_heads;
-        if (part == 0 && live)
+        if (part == 0 && head < p.n_heads)
           p.lse_part[((size_t)r * p.n_heads + head) * S + s] =
               lt > 0.f ? (m_run + log2f(lt)) * 0.69314718055994531f : -INFINITY;
-        // this thread's O: dims 256 ch + 128 half + (0..127) of head `head`
-        float* op = p.o_part + (((size_t)r * p.n_heads + head) * S + s) * MLA_D_C + 256 * ch + 128 * half;
+        // this thread's O: dims 256 ch + 128 half + (0..127) of head `head`,
+        // stored 32 dims at a time through a 4 KB [32 heads x 32 dims] tile
+        // of this warp in the P area (idle until the next unit's first
+        // probabilities, which these warps write): a store instruction then
+        // covers four whole 128-byte lines (four heads) instead of 32 pieces
+        // of 32 lines
         const uint32_t oc = tmem + lane_addr + kColO + 128 * ch;
+        uint8_t* tile = s_pbuf + (warp - kWarpSoft0) * 4096;
+        const int rd_head = lane >> 3, rd_q = lane & 7;   // reader: head 4 k + rd_head, 16-byte piece rd_q
+        const int head0 = kHPC * (int)rank + 32 * (q4 & 1);   // this warp's first head
+        const size_t head_stride = (size_t)S * MLA_D_C;         // floats between heads in o_part
+        // the reader's first head (head0 + rd_head) at dims 256 ch + 128 half + 4 rd_q
+        float* const o_rd = p.o_part + (((size_t)r * p.n_heads + head0 + rd_head) * S + s) * MLA_D_C + 256 * ch +
+                            128 * half + 4 * rd_q;
 #pragma unroll 1
         for (int c4 = 0; c4 < 4; ++c4) {
           float o[32];
           tmem_ld<32>(oc + 32 * c4, o);
           tmem_wait_ld();
-          if (live) {
-            float4* dst = reinterpret_cast<float4*>(op + 32 * c4);
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-              dst[j] = make_float4(o[4 * j] * inv_l, o[4 * j + 1] * inv_l, o[4 * j + 2] * inv_l, o[4 * j + 3] * inv_l);
+          for (int q = 0; q < 8; ++q)
+            *reinterpret_cast<float4*>(tile + lane * 128 + ((q ^ (lane & 7)) << 4)) =
+                make_float4(o[4 * q] * inv_l, o[4 * q + 1] * inv_l, o[4 * q + 2] * inv_l, o[4 * q + 3] * inv_l);
+          __syncwarp();
+          float* op = o_rd + 32 * c4;
+#pragma unroll 4
+          for (int k4 = 0; k4 < 8; ++k4, op += 4 * head_stride) {
+            const int j = 4 * k4 + rd_head;                    // head of this warp
+            if (head0 + j < p.n_heads)
+              *reinterpret_cast<float4*>(op) =
+                  *reinterpret_cast<const float4*>(tile + j * 128 + ((rd_q ^ (j & 7)) << 4));
           }
+          __syncwarp();
         }
         // this warp's part of O has been read: the pair's next unit may overwrite it
         tc_fence_before();

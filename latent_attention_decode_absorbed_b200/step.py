@@ -6,6 +6,8 @@ rope tables, workspace and outputs, as torch tensors) and runs
     mla_cache_append -> mla_absorb_q -> mla_decode_fwd -> mla_combine -> mla_out_uv
 
 on one stream.  It only allocates and marshals; every step runs in libmla.
+``DecodeStep.capture`` records the same calls as CUDA graphs, for steps whose
+device work is shorter than the host time of five marshalled calls.
 """
 from __future__ import annotations
 
@@ -105,3 +107,62 @@ class DecodeStep:
         return self.out
 
     LAUNCHES_PER_STEP = 5
+
+    # -- the step as CUDA graphs ------------------------------------------------
+    def capture(self, kv_a_new, seq_ids, positions, q_nope, q_pe, w_uk, w_uv, host_in=(), host_out=None):
+        """Record the step's five calls as three CUDA graphs on this device:
+        `pre` (append, absorb), `attend` (the split-KV decode) and `post`
+        (combine, out_uv).  A replay launches the same kernels with the same
+        arguments; the graphs read the given tensors and write `out` in place,
+        so the caller refreshes the inputs' contents before each replay.
+
+        host_in: (device tensor, pinned host tensor) pairs copied host->device
+        at the start of `pre`; host_out: a pinned host tensor that `post` ends
+        by copying `out` into.  Returns a StepGraphs."""
+        torch = self.torch
+
+        def copies_in():
+            for dst, src in host_in:
+                dst.copy_(src, non_blocking=True)
+
+        def pre():
+            copies_in()
+            self.append(kv_a_new, seq_ids, positions)
+            self.absorb(q_nope, q_pe, w_uk)
+
+        def post():
+            self.combine()
+            self.project_out(w_uv)
+            if host_out is not None:
+                host_out.copy_(self.out, non_blocking=True)
+
+        parts = (pre, self.attend, post)
+        # eager passes first (module loading, kernel attributes), on a side stream
+        side = torch.cuda.Stream(device=self.device)
+        side.wait_stream(torch.cuda.current_stream(self.device))
+        with torch.cuda.stream(side):
+            for _ in range(2):
+                for fn in parts:
+                    fn()
+        torch.cuda.current_stream(self.device).wait_stream(side)
+        torch.cuda.synchronize(self.device)
+        graphs = []
+        for fn in parts:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, capture_error_mode="thread_local"):
+                fn()
+            graphs.append(g)
+        return StepGraphs(*graphs)
+
+
+class StepGraphs:
+    """The three graphs of one captured step; `replay()` runs them in order
+    on the current stream."""
+
+    def __init__(self, pre, attend, post):
+        self.pre, self.attend, self.post = pre, attend, post
+
+    def replay(self):
+        self.pre.replay()
+        self.attend.replay()
+        self.post.replay()
