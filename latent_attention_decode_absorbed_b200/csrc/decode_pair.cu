@@ -57,24 +57,21 @@ using namespace sm100;
 constexpr int kTile = 256;                // cached rows per pair tile (128 per CTA)
 constexpr int kChunks = 9;                // 576 / 64 column chunks
 constexpr int kHPC = 64;                  // heads per CTA
-constexpr int kSlots = 7;                 // ring stages
 constexpr int kSlotBytes = 16384;         // one stage: one score chunk or one value box of this CTA
-constexpr int kBox = 8192;                // [64 rows x 64 bf16]
-constexpr int kQChunk = kHPC * 128;       // [64 heads x 64 dims] bf16
-constexpr int kPChunk = kHPC * 128;       // [64 heads x 64 rows] bf16: P of one page
+constexpr int kBox = 8192;                // [64 rows x 64 16-bit values]
+constexpr int kBox8 = 4096;               // e4m3 cache: [64 rows x 64 codes]
+constexpr int kStgBytes = 2 * kBox8;      // e4m3 cache: the raw codes of one stage
+constexpr int kQChunk = kHPC * 128;       // [64 heads x 64 dims], 16-bit
+constexpr int kPChunk = kHPC * 128;       // [64 heads x 64 rows], 16-bit: P of one page
 constexpr int kWarpProd = 0, kWarpMma = 1, kWarpSoft0 = 2, kSoftWarps = 8;
-constexpr int kThreads = 32 * (kWarpSoft0 + kSoftWarps);
+constexpr int kWarpConv0 = kWarpSoft0 + kSoftWarps, kConvWarps = 4;   // e4m3 cache: converters
 constexpr int kQN = 8;                    // unit queue depth
 constexpr float kRescaleLog2 = 8.0f;      // lazy rescale threshold (log2 units)
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;             // S of tile t at kColS + 128 (t & 1)
 constexpr uint32_t kColO = 256;           // O: dims 0..255 at 256, dims 256..511 at 384
 
-// shared memory (bytes from the 1024-aligned base)
-constexpr int kOffQ = 0;                                  // Q: 9 x 8 KB, K-major SW128
-constexpr int kOffRing = kOffQ + kChunks * kQChunk;       // ring: 7 x 16 KB
-constexpr int kOffP = kOffRing + kSlots * kSlotBytes;     // P: 4 pages x 8 KB, K-major SW128
-constexpr int kOffMisc = kOffP + 4 * kPChunk;
+// offsets inside the misc area
 constexpr int kMBars = 0;                 // 48 barriers
 constexpr int kMTmem = 48 * 8;
 constexpr int kMAbort = kMTmem + 4;
@@ -82,23 +79,43 @@ constexpr int kMRedMax = kMTmem + 16;     // float [2 tile parities][2 lane halv
 constexpr int kMRedSum = kMRedMax + 2 * 4 * kHPC * 4;   // float [2 lane halves][2 column halves][64 heads]
 constexpr int kMUnitQ = kMRedSum + 4 * kHPC * 4;
 constexpr int kMiscBytes = kMUnitQ + 4 * kQN;
-constexpr int kSmem = kOffMisc + kMiscBytes + 1024;       // + alignment slack
-static_assert(kSmem <= 227 * 1024, "shared memory budget");
 
-// barrier indices
-constexpr int kBFull = 0;                 // [kSlots] leader: both CTAs' TMA bytes of a stage
-constexpr int kBEmpty = kSlots;           // [kSlots] both: the MMAs are done with the stage
-constexpr int kBSFull = 2 * kSlots;       // [2] both: S of a tile is in TMEM
-constexpr int kBODone = kBSFull + 2;      // both: the value MMAs of a tile are done
-constexpr int kBPFull = kBODone + 1;      // leader: both CTAs' softmax wrote P (and rescaled O)
-constexpr int kBQFull = kBPFull + 1;      // leader: both CTAs' Q of the unit landed
-constexpr int kBQFree = kBQFull + 1;      // both: the unit's score MMAs are done with Q
-constexpr int kBEpiDone = kBQFree + 1;    // leader: both CTAs read O out (TMEM reusable)
-constexpr int kBUqFull = kBEpiDone + 1;   // [kQN] both: unit queue slot written
-constexpr int kBUqEmpty = kBUqFull + kQN; // [kQN] leader: every consumer read the slot
-constexpr int kBSoft = kBUqEmpty + kQN;   // [2] local: the softmax warps' own barriers (bounded waits)
-constexpr int kBEnd = kBSoft + 2;
-static_assert(kBEnd <= 48, "barrier area");
+// Shared memory, barriers and threads of the bf16 (F8 = false) and e4m3
+// (F8 = true) kernels.  With an e4m3 cache the producer's copies land in a
+// staging ring of raw codes and four converter warps widen them into the
+// operand ring (one slot fewer, to make room for the staging).
+template <bool F8>
+struct PairLayout {
+  static constexpr int kSlots = F8 ? kConvWarps : 7;      // operand ring stages (e4m3: one per converter)
+  static constexpr int kStg = F8 ? 6 : 0;                 // staging slots
+  static constexpr int kThreads = 32 * (kWarpSoft0 + kSoftWarps + (F8 ? kConvWarps : 0));
+  // bytes from the 1024-aligned base
+  static constexpr int kOffQ = 0;                          // Q: 9 x 8 KB, K-major SW128
+  static constexpr int kOffRing = kOffQ + kChunks * kQChunk;
+  static constexpr int kOffP = kOffRing + kSlots * kSlotBytes;   // P: 4 pages x 8 KB, K-major SW128
+  static constexpr int kOffStg = kOffP + 4 * kPChunk;
+  static constexpr int kOffMisc = kOffStg + kStg * kStgBytes;
+  static constexpr int kSmem = kOffMisc + kMiscBytes + 1024;     // + alignment slack
+  // barrier indices
+  static constexpr int kBFull = 0;                  // [kSlots] leader: a stage is in both CTAs (TMA
+                                                    // bytes; e4m3: the stage's converter warp of each CTA)
+  static constexpr int kBEmpty = kSlots;            // [kSlots] both: the MMAs are done with the stage
+  static constexpr int kBSFull = 2 * kSlots;        // [2] both: S of a tile is in TMEM
+  static constexpr int kBODone = kBSFull + 2;       // both: the value MMAs of a tile are done
+  static constexpr int kBPFull = kBODone + 1;       // leader: both CTAs' softmax wrote P (and rescaled O)
+  static constexpr int kBQFull = kBPFull + 1;       // bf16: leader, both CTAs' Q landed; e4m3: local
+  static constexpr int kBQFree = kBQFull + 1;       // both: the unit's score MMAs are done with Q
+  static constexpr int kBEpiDone = kBQFree + 1;     // leader: both CTAs read O out (TMEM reusable)
+  static constexpr int kBUqFull = kBEpiDone + 1;    // [kQN] both: unit queue slot written
+  static constexpr int kBUqEmpty = kBUqFull + kQN;  // [kQN] leader: every consumer read the slot
+  static constexpr int kBSoft = kBUqEmpty + kQN;    // [2] local: the softmax warps' own barriers
+  static constexpr int kBStgFull = kBSoft + 2;      // [kStg] local: raw codes landed
+  static constexpr int kBStgEmpty = kBStgFull + kStg;   // [kStg] local: the converters read them
+  static constexpr int kBQReady = kBStgEmpty + kStg;    // leader: both CTAs' Q widened to f16
+  static constexpr int kBEnd = kBQReady + 1;
+  static_assert(kSmem <= 227 * 1024, "shared memory budget");
+  static_assert(kBEnd <= 48, "barrier area");
+};
 
 struct PairParams {
   int n_heads, q_len, batch;
@@ -115,6 +132,7 @@ struct PairParams {
   int32_t* err;
   unsigned long long wait_limit;
   int withhold_q;
+  const float* cache_scale;    // e4m3 cache: per-row dequantisation scale [num_pages * 64]
 };
 
 // page id of a cached row of sequence b (0 for rows outside the table or the
@@ -135,11 +153,27 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&v);
 }
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+  const __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+// tm_cache: boxes of one [64 rows x 64 columns] block (e4m3: [64 x 64 codes]);
+// tm_cache2: boxes of two adjacent blocks (bf16 only); tm_q: q_abs boxes.
+template <bool F8>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<F8>::kThreads, 1)
     decode_pair_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_constant__ CUtensorMap tm_cache2,
                        const __grid_constant__ CUtensorMap tm_q, const PairParams p) {
-  constexpr int kQConsumers = 2 + 2 * kSoftWarps;   // peer producer, MMA warp, softmax warps of both CTAs
+  using L = PairLayout<F8>;
+  constexpr int kSlots = L::kSlots, kStg = L::kStg;
+  constexpr int kOffQ = L::kOffQ, kOffRing = L::kOffRing, kOffP = L::kOffP, kOffStg = L::kOffStg,
+                kOffMisc = L::kOffMisc;
+  constexpr int kBFull = L::kBFull, kBEmpty = L::kBEmpty, kBSFull = L::kBSFull, kBODone = L::kBODone,
+                kBPFull = L::kBPFull, kBQFull = L::kBQFull, kBQFree = L::kBQFree, kBEpiDone = L::kBEpiDone,
+                kBUqFull = L::kBUqFull, kBUqEmpty = L::kBUqEmpty, kBSoft = L::kBSoft, kBStgFull = L::kBStgFull,
+                kBStgEmpty = L::kBStgEmpty, kBQReady = L::kBQReady;
+  // queue readers: peer producer, MMA warp, softmax (and converter) warps of both CTAs
+  constexpr int kQConsumers = 2 + 2 * kSoftWarps + (F8 ? 2 * kConvWarps : 0);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t s_base = smem_u32(smem);
@@ -194,9 +228,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (leader && threadIdx.x == 0) first_claim = atomicAdd(p.claim, 1u);
   if (threadIdx.x == 0) {
     for (int i = 0; i < kSlots; ++i) {
-      mbar_init(bar(kBFull + i), 1);
+      mbar_init(bar(kBFull + i), F8 ? 2 : 1);
       mbar_init(bar(kBEmpty + i), 1);
     }
+    for (int i = 0; i < kStg; ++i) {
+      mbar_init(bar(kBStgFull + i), 1);
+      mbar_init(bar(kBStgEmpty + i), 1);
+    }
+    if (F8) mbar_init(bar(kBQReady), 2 * kConvWarps);
     mbar_init(bar(kBSFull), 1);
     mbar_init(bar(kBSFull + 1), 1);
     mbar_init(bar(kBODone), 1);
@@ -247,12 +286,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // S(0), then per tile i: S(i+1), O(i).  The pool is page-blocked (nine
     // contiguous [64 rows x 64 columns] blocks per page), viewed as 2-D
     // [blocks * 64 lines x 64 columns].  A score stage is column chunk c of
-    // this CTA's two pages of the tile (lane l < 2: block c of page l, 8 KB);
+    // this CTA's two pages of the tile (block c of each page, 8 KB each);
     // a value stage is one page's pair of dims blocks 4 bb + 2 r, +1 of this
-    // CTA (one contiguous 16 KB box).
+    // CTA (one contiguous 16 KB box).  e4m3 cache: the same blocks as raw
+    // codes (4 KB each) into a staging slot of this CTA, for the converters.
     if (lane == 0) {
       tma_prefetch_desc(&tm_cache);
-      tma_prefetch_desc(&tm_cache2);
+      if (!F8) tma_prefetch_desc(&tm_cache2);
       tma_prefetch_desc(&tm_q);
     }
     // score rows are re-read by the value stages of the pair (this CTA's for
@@ -285,10 +325,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // (test hook: the leader leaves the query load of its first unit out,
         // so the MMA issuer's wait for it runs out and the launch aborts)
         if (ok && !(p.withhold_q && leader && uc == 0)) {
-          const uint32_t q_bar = mapa(bar(kBQFull), 0);
-          if (leader) mbar_arrive_expect_tx(bar(kBQFull), 2u * kChunks * kQChunk);
-          for (int c = 0; c < kChunks; ++c)
-            tma_load_3d_pair(s_q + c * kQChunk, &tm_q, 64 * c, (int)rank * kHPC, r, q_bar);
+          if constexpr (F8) {
+            // each CTA's half lands on its own barrier; the converters widen it to f16
+            mbar_arrive_expect_tx(bar(kBQFull), kChunks * kQChunk);
+            for (int c = 0; c < kChunks; ++c)
+              tma_load_3d(s_q + c * kQChunk, &tm_q, 64 * c, (int)rank * kHPC, r, bar(kBQFull));
+          } else {
+            const uint32_t q_bar = mapa(bar(kBQFull), 0);
+            if (leader) mbar_arrive_expect_tx(bar(kBQFull), 2u * kChunks * kQChunk);
+            for (int c = 0; c < kChunks; ++c)
+              tma_load_3d_pair(s_q + c * kQChunk, &tm_q, 64 * c, (int)rank * kHPC, r, q_bar);
+          }
         }
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -304,12 +351,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // rows outside the table or the pool read page 0 (readable; they are masked)
         auto page = [&](int pg) -> int { return pg >= 0 && pg < p.num_pages ? pg : 0; };
         auto take = [&](uint32_t& dst, uint32_t& fb) -> bool {
-          const uint32_t slot = kc % kSlots;
-          const uint32_t ph = (kc / kSlots) & 1u;
-          if (!mbar_wait<false>(bar(kBEmpty + slot), ph ^ 1u, abort_flag, lim)) return false;
-          if (leader) mbar_arrive_expect_tx(bar(kBFull + slot), 2u * kSlotBytes);
-          dst = s_ring + slot * kSlotBytes;
-          fb = mapa(bar(kBFull + slot), 0);
+          if constexpr (F8) {
+            const uint32_t slot = kc % kStg;
+            const uint32_t ph = (kc / kStg) & 1u;
+            if (!mbar_wait<false>(bar(kBStgEmpty + slot), ph ^ 1u, abort_flag, lim)) return false;
+            mbar_arrive_expect_tx(bar(kBStgFull + slot), kStgBytes);
+            dst = s_base + kOffStg + slot * kStgBytes;
+            fb = bar(kBStgFull + slot);
+          } else {
+            const uint32_t slot = kc % kSlots;
+            const uint32_t ph = (kc / kSlots) & 1u;
+            if (!mbar_wait<false>(bar(kBEmpty + slot), ph ^ 1u, abort_flag, lim)) return false;
+            if (leader) mbar_arrive_expect_tx(bar(kBFull + slot), 2u * kSlotBytes);
+            dst = s_ring + slot * kSlotBytes;
+            fb = mapa(bar(kBFull + slot), 0);
+          }
           ++kc;
           return true;
         };
@@ -318,8 +374,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           for (int c = 0; c < kChunks; ++c) {
             uint32_t dst, fb;
             if (!take(dst, fb)) return false;
-            tma_load_2d_pair_hint(dst, &tm_cache, 0, (pg0 * kChunks + c) * 64, fb, pol_keep);
-            tma_load_2d_pair_hint(dst + kBox, &tm_cache, 0, (pg1 * kChunks + c) * 64, fb, pol_keep);
+            if constexpr (F8) {
+              tma_load_2d_hint(dst, &tm_cache, 0, (pg0 * kChunks + c) * 64, fb, pol_keep);
+              tma_load_2d_hint(dst + kBox8, &tm_cache, 0, (pg1 * kChunks + c) * 64, fb, pol_keep);
+            } else {
+              tma_load_2d_pair_hint(dst, &tm_cache, 0, (pg0 * kChunks + c) * 64, fb, pol_keep);
+              tma_load_2d_pair_hint(dst + kBox, &tm_cache, 0, (pg1 * kChunks + c) * 64, fb, pol_keep);
+            }
           }
           return true;
         };
@@ -331,8 +392,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             for (int bb = 0; bb < 2; ++bb) {
               uint32_t dst, fb;
               if (!take(dst, fb)) return false;
-              tma_load_2d_pair_hint(dst, &tm_cache2, 0, (pg[pg_i] * kChunks + 4 * bb + 2 * (int)rank) * 64, fb,
-                                    pol_drop);
+              const int line = (pg[pg_i] * kChunks + 4 * bb + 2 * (int)rank) * 64;
+              if constexpr (F8) {
+                tma_load_2d_hint(dst, &tm_cache, 0, line, fb, pol_drop);
+                tma_load_2d_hint(dst + kBox8, &tm_cache, 0, line + 64, fb, pol_drop);
+              } else {
+                tma_load_2d_pair_hint(dst, &tm_cache2, 0, line, fb, pol_drop);
+              }
             }
           }
           return true;
@@ -374,12 +440,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // O(i-1) is done (one P buffer), so running the score GEMM further ahead
     // only delays O(i) (measured slower).
     if (leader) {
-      constexpr uint32_t idS = idesc_f16(128, 256, false, false);
-      constexpr uint32_t idO = idesc_f16(128, 256, false, true);
+      // e4m3 cache: the operands are f16 (widened codes, Q and P in f16)
+      constexpr uint32_t idS = idesc_f16(128, 256, false, false, F8);
+      constexpr uint32_t idO = idesc_f16(128, 256, false, true, F8);
       auto ready = [&](uint32_t& src, uint32_t& empty) -> bool {
         const uint32_t slot = kc % kSlots;
         const uint32_t ph = (kc / kSlots) & 1u;
-        if (!__all_sync(0xffffffffu, mbar_wait<false>(bar(kBFull + slot), ph, abort_flag, lim))) return false;
+        // e4m3: the converters' arrivals carry generic writes of both CTAs (cluster scope)
+        if (!__all_sync(0xffffffffu, mbar_wait<F8>(bar(kBFull + slot), ph, abort_flag, lim))) return false;
         tc_fence_after();
         src = s_ring + slot * kSlotBytes;
         empty = bar(kBEmpty + slot);
@@ -398,7 +466,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         f += U.s1 - U.s;
         if (U.n_tiles == 0) continue;
         const int lo = U.lo, hi = U.hi, n_tiles = U.n_tiles;
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(kBQFull), uc & 1, abort_flag, lim));
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(F8 ? kBQReady : kBQFull), uc & 1, abort_flag, lim));
         if (!ok) break;
         tc_fence_after();
         auto issue_s = [&](int i) -> bool {
@@ -456,7 +524,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else {
+  } else if (warp < kWarpConv0) {
     // ================= softmax (both CTAs, warps 2-9) =================
     // Thread (lane quadrant q4, column half ch, lane) owns head hh = 32 (q4 & 1)
     // + lane of this CTA and the 64 tile rows 128 (q4 >> 1) + 64 ch .. +63.
@@ -506,12 +574,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // read before the wait for the scores, off the critical path)
         const int row0 = lo + kTile * i + 128 * half + 64 * ch;
         int nvalid = min(max(hi - row0, 0), 64);
+        float sc_lo = 1.f, sc_hi = 1.f;   // e4m3: the page's dequantisation scales (lane l: rows l, l + 32)
         if (nvalid > 0) {
           bool pok;
-          (void)page_of(p, b, row0, &pok);
+          const int pg = page_of(p, b, row0, &pok);
           if (!pok) {
             nvalid = 0;
             flag_error(p.err, MLA_DEVERR_PAGE);
+          } else if constexpr (F8) {
+            sc_lo = __ldg(p.cache_scale + (size_t)pg * 64 + lane);
+            sc_hi = __ldg(p.cache_scale + (size_t)pg * 64 + 32 + lane);
           }
         }
         ok = __all_sync(0xffffffffu, mbar_wait<false>(bar(kBSFull + sb), (t >> 1) & 1, abort_flag, lim));
@@ -525,7 +597,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         float mx = -INFINITY;
 #pragma unroll
         for (int j = 0; j < 64; ++j) {
-          v[j] = j < nvalid ? v[j] * p.scale_log2 : -INFINITY;
+          float sl = p.scale_log2;
+          if constexpr (F8) sl *= __shfl_sync(0xffffffffu, j < 32 ? sc_lo : sc_hi, j & 31);
+          v[j] = j < nvalid ? v[j] * sl : -INFINITY;
           mx = fmaxf(mx, v[j]);
         }
         // the four partial maxima of each head, double-buffered by tile parity:
@@ -547,7 +621,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int j = 0; j < 32; ++j) {
           const float p0 = exp2_approx(v[2 * j] - msub), p1 = exp2_approx(v[2 * j + 1] - msub);
           sum += p0 + p1;
-          pk[j] = pack_bf16(p0, p1);
+          pk[j] = F8 ? pack_f16(p0, p1) : pack_bf16(p0, p1);
         }
         l_acc = changed ? fmaf(l_acc, alpha, sum) : l_acc + sum;
         // every phase of o_done is observed in order (a parity wait cannot
@@ -642,6 +716,121 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       ++uc;
       }
     }
+  } else {
+    // ============ e4m3 -> f16 converters (both CTAs, warps 10-13) ============
+    // Per segment: Q (bf16 -> f16 in place, all four warps), then the stages
+    // in the MMA's order, dealt round robin: warp w converts stages w, w + 4,
+    // ... into operand slot w.  For its stage a warp waits for the staging
+    // slot's codes and the operand slot's release, widens the codes exactly
+    // (every e4m3 value is an f16 value), writes them 128-byte swizzled like
+    // the bf16 copies, makes them visible to the tensor core and arrives on
+    // the leader's full barrier.  Value stages are also multiplied by the
+    // row's dequantisation scale (an f16 product); scores get the scale in
+    // the softmax instead.
+    if constexpr (F8) {
+      const int cw = warp - kWarpConv0;               // 0..3
+      const int ct = threadIdx.x - 32 * kWarpConv0;   // 0..127
+      constexpr int kCT = 32 * kConvWarps;
+      uint32_t uc = 0;
+      bool ok = true;
+      for (uint32_t k = 0; ok; ++k) {
+        const int u = next_unit(k);
+        if (u == -2) { ok = false; break; }
+        if (u < 0) break;
+        const int f1 = min(n_flat, (u + 1) * p.run);
+        for (int f = u * p.run; f < f1 && ok;) {
+        const UnitInfo U = seg_at(f, f1);
+        f += U.s1 - U.s;
+        if (U.n_tiles == 0) continue;
+        const int b = U.b, lo = U.lo, hi = U.hi, n_tiles = U.n_tiles;
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait<false>(bar(kBQFull), uc & 1, abort_flag, lim)))) break;
+        for (int i = ct; i < kChunks * kQChunk / 16; i += kCT) {
+          uint4 v = *reinterpret_cast<const uint4*>(smem + kOffQ + 16 * i);
+          uint32_t* w = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+            w[e] = pack_f16(f2.x, f2.y);
+          }
+          *reinterpret_cast<uint4*>(smem + kOffQ + 16 * i) = v;
+        }
+        fence_proxy_async_cta();     // read by the tensor core
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(mapa(bar(kBQReady), 0));
+        // one stage: two [64 x 64] blocks of codes -> two [64 x 64] f16 blocks;
+        // lane l handles 16 codes of rows (l >> 2) + 8 i, i = 0..15 (8 per block)
+        auto convert = [&](int scale_page) -> bool {
+          const uint32_t my = kc++;
+          if ((int)(my % kConvWarps) != cw) return true;   // another warp's stage
+          const uint32_t slot = my % kSlots, ph = (my / kSlots) & 1u;
+          const uint32_t ss = my % kStg, sph = (my / kStg) & 1u;
+          // value stage: lane l holds the scales of rows l and l + 32 of the page
+          float s_lo = 1.f, s_hi = 1.f;
+          if (scale_page >= 0) {
+            s_lo = __ldg(p.cache_scale + (size_t)scale_page * 64 + lane);
+            s_hi = __ldg(p.cache_scale + (size_t)scale_page * 64 + 32 + lane);
+          }
+          if (!__all_sync(0xffffffffu, mbar_wait<false>(bar(kBStgFull + ss), sph, abort_flag, lim))) return false;
+          if (!__all_sync(0xffffffffu, mbar_wait<false>(bar(kBEmpty + slot), ph ^ 1u, abort_flag, lim))) return false;
+          const uint8_t* src = smem + kOffStg + ss * kStgBytes;
+          uint8_t* dst = smem + kOffRing + slot * kSlotBytes;
+          const int qq = lane & 3;
+#pragma unroll 4
+          for (int i = 0; i < 16; ++i) {
+            const int box = i >> 3, row = (lane >> 2) + 8 * (i & 7);
+            const uint4 codes = *reinterpret_cast<const uint4*>(src + box * kBox8 + row * 64 + qq * 16);
+            const uint32_t* cwd = reinterpret_cast<const uint32_t*>(&codes);
+            const float sr = __shfl_sync(0xffffffffu, row < 32 ? s_lo : s_hi, row & 31);
+            const __half2 rs2 = __float2half2_rn(sr);
+            uint32_t hw[8];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+#pragma unroll
+              for (int hf = 0; hf < 2; ++hf) {
+                const __half2_raw r2 = __nv_cvt_fp8x2_to_halfraw2(
+                    static_cast<__nv_fp8x2_storage_t>((cwd[e] >> (16 * hf)) & 0xffffu), __NV_E4M3);
+                __half2 h2 = *reinterpret_cast<const __half2*>(&r2);
+                if (scale_page >= 0) h2 = __hmul2(h2, rs2);
+                hw[2 * e + hf] = *reinterpret_cast<const uint32_t*>(&h2);
+              }
+            }
+            uint8_t* rowp = dst + box * kBox + row * 128;
+            *reinterpret_cast<uint4*>(rowp + (((2 * qq) ^ (row & 7)) << 4)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+            *reinterpret_cast<uint4*>(rowp + (((2 * qq + 1) ^ (row & 7)) << 4)) = make_uint4(hw[4], hw[5], hw[6], hw[7]);
+          }
+          fence_proxy_async_cta();     // read by the tensor core
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive_cluster(mapa(bar(kBFull + slot), 0));
+            mbar_arrive_local(bar(kBStgEmpty + ss));
+          }
+          return true;
+        };
+        auto conv_s = [&]() -> bool {
+          for (int c = 0; c < kChunks; ++c)
+            if (!convert(-1)) return false;
+          return true;
+        };
+        auto conv_o = [&](int j) -> bool {
+          for (int pg_i = 0; pg_i < 4; ++pg_i) {
+            const int row0 = lo + kTile * j + 64 * pg_i;
+            if (row0 >= hi) break;
+            bool vld;
+            const int pg = page_of(p, b, row0, &vld);
+            for (int bb = 0; bb < 2; ++bb)
+              if (!convert(pg)) return false;
+          }
+          return true;
+        };
+        ok = conv_s();
+        for (int i = 0; i < n_tiles && ok; ++i) {
+          if (i + 1 < n_tiles) ok = conv_s();
+          if (ok) ok = conv_o(i);
+        }
+        ++uc;
+        }
+      }
+    }
   }
 
   // ---- teardown
@@ -702,25 +891,40 @@ bool claim_slot(const void* workspace, unsigned** claim, unsigned** done) {
 }  // namespace
 
 bool decode_pair_supported(const DecodeArgs& a) {
-  return a.q_dtype == MLA_BF16 && a.cache_dtype == MLA_BF16 && a.page_size == 64 && a.n_heads > 64 &&
-         a.n_heads <= 128 && (long long)a.batch * a.q_len * a.num_splits * 2 < (1ll << 31);
+  return a.q_dtype == MLA_BF16 && (a.cache_dtype == MLA_BF16 || a.cache_dtype == MLA_E4M3) && a.page_size == 64 &&
+         a.n_heads > 64 && a.n_heads <= 128 && (long long)a.batch * a.q_len * a.num_splits * 2 < (1ll << 31);
 }
 
 cudaError_t launch_decode_pair(const DecodeArgs& a, cudaStream_t st) {
   TensorMapEncodeFn enc = tensor_map_encoder();
   if (!enc) return cudaErrorNotSupported;
+  const bool f8 = a.cache_dtype == MLA_E4M3;
   CUtensorMap tc, tc2, tq;
-  // the page-blocked pool as 2-D [num_pages * 9 * 64 lines x 64 columns] of
-  // 128-byte lines: boxes of 64 lines (one block) and 128 lines (two adjacent blocks)
-  for (int k = 0; k < 2; ++k) {
+  if (f8) {
+    // the e4m3 pool as 2-D [num_pages * 9 * 64 lines x 64 codes] of 64-byte
+    // lines, unswizzled (the converters swizzle): boxes of one block
     cuuint64_t dims[2] = {64, (cuuint64_t)a.num_pages * kChunks * 64};
-    cuuint64_t strides[1] = {128};
-    cuuint32_t box[2] = {64, k == 0 ? 64u : 128u};
+    cuuint64_t strides[1] = {64};
+    cuuint32_t box[2] = {64, 64};
     cuuint32_t es[2] = {1, 1};
-    if (enc(k == 0 ? &tc : &tc2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a.cache), dims, strides, box,
-            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+    if (enc(&tc, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(a.cache), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
+    tc2 = tc;
+  } else {
+    // the page-blocked pool as 2-D [num_pages * 9 * 64 lines x 64 columns] of
+    // 128-byte lines: boxes of 64 lines (one block) and 128 lines (two adjacent blocks)
+    for (int k = 0; k < 2; ++k) {
+      cuuint64_t dims[2] = {64, (cuuint64_t)a.num_pages * kChunks * 64};
+      cuuint64_t strides[1] = {128};
+      cuuint32_t box[2] = {64, k == 0 ? 64u : 128u};
+      cuuint32_t es[2] = {1, 1};
+      if (enc(k == 0 ? &tc : &tc2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a.cache), dims, strides,
+              box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    }
   }
   {
     // q_abs [rows, heads, 576]: boxes of 64 columns x 64 heads of one row
@@ -734,7 +938,9 @@ cudaError_t launch_decode_pair(const DecodeArgs& a, cudaStream_t st) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  cudaError_t e = cudaFuncSetAttribute(decode_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+  const int smem = f8 ? PairLayout<true>::kSmem : PairLayout<false>::kSmem;
+  cudaError_t e = f8 ? cudaFuncSetAttribute(decode_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)
+                     : cudaFuncSetAttribute(decode_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   // Runs of splits per claimed unit.  With at least four splits per CTA pair,
   // every pair gets one run of ceil(splits / pairs) consecutive splits: each
@@ -749,10 +955,13 @@ cudaError_t launch_decode_pair(const DecodeArgs& a, cudaStream_t st) {
   const long long units = (n_flat + run - 1) / run;
   PairParams p{a.n_heads, a.q_len, a.batch, a.block_table, a.max_pages, a.num_pages, a.seq_lens, a.num_splits,
                a.split_tokens, run, a.softmax_scale * 1.4426950408889634f, nullptr, nullptr, a.o_part, a.lse_part,
-               a.err, g_wait_limit.load(), g_withhold_q.load()};
+               a.err, g_wait_limit.load(), g_withhold_q.load(), a.cache_scale};
   if (!claim_slot(a.o_part, &p.claim, &p.done)) return cudaErrorInvalidSymbol;
   const long long pairs = units < P ? units : P;
-  decode_pair_kernel<<<dim3((unsigned)(2 * pairs)), kThreads, kSmem, st>>>(tc, tc2, tq, p);
+  if (f8)
+    decode_pair_kernel<true><<<dim3((unsigned)(2 * pairs)), PairLayout<true>::kThreads, smem, st>>>(tc, tc2, tq, p);
+  else
+    decode_pair_kernel<false><<<dim3((unsigned)(2 * pairs)), PairLayout<false>::kThreads, smem, st>>>(tc, tc2, tq, p);
   return cudaGetLastError();
 }
 

@@ -216,6 +216,10 @@ CASES = [
     ("heads16_many_splits_e4m3", "e4m3", [700], 1, 16, 64),
     ("multi_tile_e4m3", "e4m3", [1100, 600], 2, 128, 1024),
     ("long_split_e4m3", "e4m3", [5000], 1, 128, 4096),
+    # the e4m3 cache on the head-split pair: padded heads, two tokens, merged runs
+    ("heads96_mtp_e4m3", "e4m3", [700, 65, 2], 2, 96, 128),
+    ("heads65_e4m3", "e4m3", [129], 1, 65, 64),
+    ("many_units_mtp_e4m3", "e4m3", [1500] * 6 + [7000], 2, 128, 128),
     ("tiny_f32", "f32", [256, 37], 1, 16, 64),
 ]
 
