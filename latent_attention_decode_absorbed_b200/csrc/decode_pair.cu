@@ -40,7 +40,15 @@
 //
 // Warp roles per CTA: 0 TMA producer and TMEM allocator, 1 MMA issuer (the
 // leader CTA issues for the pair), 2-9 softmax (warp w reads TMEM lanes
-// 32 (w % 4) .. +31; warps 2-5 take score columns 0-63, warps 6-9 64-127).
+// 32 (w % 4) .. +31; warps 2-5 take score columns 0-63, warps 6-9 64-127),
+// and with an e4m3 cache 10-13 converters (codes -> f16 operands).
+//
+// Hand-offs of shared-memory operands to the MMA issuer (P, and with an
+// e4m3 cache Q and the widened stages) arrive on the leader's barriers with
+// a CTA-scope release after a proxy fence: each CTA's half of a cta_group::2
+// MMA reads that CTA's own shared memory on its own SM, so the leader only
+// needs to know when to issue.  A cluster-scope release there stalled the
+// arriving warp ~1.2K cycles (the e4m3 launch: 570 -> 425 us).
 #include <math.h>
 
 #include <mutex>
@@ -446,8 +454,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<F8>::kThr
       auto ready = [&](uint32_t& src, uint32_t& empty) -> bool {
         const uint32_t slot = kc % kSlots;
         const uint32_t ph = (kc / kSlots) & 1u;
-        // e4m3: the converters' arrivals carry generic writes of both CTAs (cluster scope)
-        if (!__all_sync(0xffffffffu, mbar_wait<F8>(bar(kBFull + slot), ph, abort_flag, lim))) return false;
+        if (!__all_sync(0xffffffffu, mbar_wait<false>(bar(kBFull + slot), ph, abort_flag, lim))) return false;
         tc_fence_after();
         src = s_ring + slot * kSlotBytes;
         empty = bar(kBEmpty + slot);
@@ -466,7 +473,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<F8>::kThr
         f += U.s1 - U.s;
         if (U.n_tiles == 0) continue;
         const int lo = U.lo, hi = U.hi, n_tiles = U.n_tiles;
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(F8 ? kBQReady : kBQFull), uc & 1, abort_flag, lim));
+        ok = __all_sync(0xffffffffu, mbar_wait<false>(bar(F8 ? kBQReady : kBQFull), uc & 1, abort_flag, lim));
         if (!ok) break;
         tc_fence_after();
         auto issue_s = [&](int i) -> bool {
@@ -490,7 +497,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<F8>::kThr
         };
         auto issue_o = [&](int j) -> bool {
           const uint32_t t = gt + j;
-          if (!__all_sync(0xffffffffu, mbar_wait(bar(kBPFull), t & 1, abort_flag, lim))) return false;
+          if (!__all_sync(0xffffffffu, mbar_wait<false>(bar(kBPFull), t & 1, abort_flag, lim))) return false;
           // the accumulator is overwritten by this unit's first value MMA: the
           // previous unit's epilogue must have read it out
           if (j == 0 && uc > 0 &&
@@ -658,7 +665,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<F8>::kThr
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(mapa(bar(kBPFull), 0));
+        if (lane == 0) mbar_arrive_cluster_cta(mapa(bar(kBPFull), 0));
       }
       // ---- epilogue: normalise O by the row sums, write o_part and lse
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait<false>(bar(kBODone), (gt + n_tiles - 1) & 1, abort_flag, lim));
@@ -756,7 +763,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<F8>::kThr
         }
         fence_proxy_async_cta();     // read by the tensor core
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(mapa(bar(kBQReady), 0));
+        if (lane == 0) mbar_arrive_cluster_cta(mapa(bar(kBQReady), 0));
         // one stage: two [64 x 64] blocks of codes -> two [64 x 64] f16 blocks;
         // lane l handles 16 codes of rows (l >> 2) + 8 i, i = 0..15 (8 per block)
         auto convert = [&](int scale_page) -> bool {
@@ -801,7 +808,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<F8>::kThr
           fence_proxy_async_cta();     // read by the tensor core
           __syncwarp();
           if (lane == 0) {
-            mbar_arrive_cluster(mapa(bar(kBFull + slot), 0));
+            mbar_arrive_cluster_cta(mapa(bar(kBFull + slot), 0));
             mbar_arrive_local(bar(kBStgEmpty + ss));
           }
           return true;
