@@ -50,13 +50,23 @@ __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ 
   sum = red[0] + red[1] + red[2] + red[3];
   const float inv = sum > 0.f ? 1.0f / sum : 0.f;
   const float4* op = reinterpret_cast<const float4*>(o_part + rh * st.o_rh) + threadIdx.x;
+  const size_t ps = st.o_part / 4;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s = 0; s < S; ++s) {
-    const float ws = w[s];
-    if (ws == 0.f) continue;
-    const float4 v = op[(size_t)s * (st.o_part / 4)];
-    acc.x = fmaf(ws, v.x, acc.x); acc.y = fmaf(ws, v.y, acc.y);
-    acc.z = fmaf(ws, v.z, acc.z); acc.w = fmaf(ws, v.w, acc.w);
+  // eight parts per batch: their loads are issued together, so a batch costs
+  // one memory latency (parts of weight 0 are not read: their o may be unset)
+  for (int s0 = 0; s0 < S; s0 += 8) {
+    float ws[8];
+    float4 v[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      ws[k] = s0 + k < S ? w[s0 + k] : 0.f;
+      v[k] = ws[k] != 0.f ? op[(size_t)(s0 + k) * ps] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      acc.x = fmaf(ws[k], v[k].x, acc.x); acc.y = fmaf(ws[k], v[k].y, acc.y);
+      acc.z = fmaf(ws[k], v[k].z, acc.z); acc.w = fmaf(ws[k], v[k].w, acc.w);
+    }
   }
   OT* dst = o_lat + rh * MLA_D_C + 4 * threadIdx.x;
   dst[0] = from_f32<OT>(acc.x * inv); dst[1] = from_f32<OT>(acc.y * inv);
