@@ -233,6 +233,17 @@ def stored_rows(rows: np.ndarray, cache_dtype: str):
 # --------------------------------------------------------------------------
 # attention, naive form  [V2-C] §1-§3 (Appendix C formulas)
 # --------------------------------------------------------------------------
+def decompress_kv(c_hat, w_uk, w_uv):
+    """Per-head keys and values of cached latents, [V2-C] §2 ("up-project"):
+    k^C_{j,i} = W^UK_i c_j and v^C_{j,i} = W^UV_i c_j.  c_hat [L, 512],
+    w_uk / w_uv [H, 128, 512]; returns k_c, v_c [L, H, 128].  This is the
+    "decompress" step of the non-absorbed (level 2) decode."""
+    c_hat = np.asarray(c_hat, np.float64)
+    k_c = np.einsum("lc,hkc->lhk", c_hat, np.asarray(w_uk, np.float64))
+    v_c = np.einsum("lc,hkc->lhk", c_hat, np.asarray(w_uv, np.float64))
+    return k_c, v_c
+
+
 def attention_naive(q_nope, q_pe, w_uk, w_uv, c_hat, k_r, softmax_scale=None):
     """Per-head output o_{t,i} of one sequence, naive form.
 
@@ -251,9 +262,9 @@ def attention_naive(q_nope, q_pe, w_uk, w_uv, c_hat, k_r, softmax_scale=None):
     L = c_hat.shape[0]
     scale = 1.0 / math.sqrt(D_N + D_R) if softmax_scale is None else softmax_scale
     out = np.zeros((T, H, D_V))
+    k_all, v_all = decompress_kv(c_hat, w_uk, w_uv)  # [L, H, 128]: row j = W^UK_i c_j, W^UV_i c_j
     for i in range(H):
-        k_c = c_hat @ w_uk[i].T                      # [L, 128]: row j = W^UK_i c_j
-        v_c = c_hat @ w_uv[i].T                      # [L, 128]: row j = W^UV_i c_j
+        k_c, v_c = k_all[:, i], v_all[:, i]
         k = np.concatenate([k_c, k_r], axis=1)       # [L, 192]
         for t in range(T):
             n_vis = L - T + t + 1

@@ -395,7 +395,39 @@ def pin_kv_a_projection():
     np.testing.assert_allclose(pn(rows[:, 512:]), pn(kv[:, 512:]), rtol=1e-13)
 
 
+def pin_decompress_kv():
+    """k^C = W^UK c, v^C = W^UV c per head: one-hot rows of W pick single
+    latent components; W^UK and W^UV are not swapped; scalar loops agree."""
+    g = _rng(83)
+    L, H = 3, 2
+    c = g.standard_normal((L, 512))
+    w_uk = np.zeros((H, 128, 512))
+    w_uv = np.zeros((H, 128, 512))
+    # head h, output i picks latent component (7 i + h) mod 512 for keys, (5 i + 3 h + 1) mod 512 for values
+    for h in range(H):
+        for i in range(128):
+            w_uk[h, i, (7 * i + h) % 512] = 1.0
+            w_uv[h, i, (5 * i + 3 * h + 1) % 512] = 1.0
+    k_c, v_c = oracle.decompress_kv(c, w_uk, w_uv)
+    assert k_c.shape == (L, H, 128) and v_c.shape == (L, H, 128)
+    for h in range(H):
+        for i in range(128):
+            np.testing.assert_array_equal(k_c[:, h, i], c[:, (7 * i + h) % 512])
+            np.testing.assert_array_equal(v_c[:, h, i], c[:, (5 * i + 3 * h + 1) % 512])
+    # scalar loops with dense weights
+    w_uk = g.standard_normal((H, 128, 512)) / 20
+    w_uv = g.standard_normal((H, 128, 512)) / 20
+    k_c, v_c = oracle.decompress_kv(c, w_uk, w_uv)
+    for j in range(L):
+        for h in range(H):
+            for i in (0, 63, 127):
+                rk = sum(w_uk[h, i, m] * c[j, m] for m in range(512))
+                rv = sum(w_uv[h, i, m] * c[j, m] for m in range(512))
+                assert abs(k_c[j, h, i] - rk) <= 1e-12 * (1 + abs(rk))
+                assert abs(v_c[j, h, i] - rv) <= 1e-12 * (1 + abs(rv))
+
+
 ALL_PINS = [pin_cache_arithmetic, pin_rmsnorm, pin_rope, pin_e4m3, pin_bf16_rounding,
             pin_naive_equals_absorbed, pin_single_row, pin_uniform_scores, pin_two_rows_sigmoid,
             pin_row_permutation, pin_causal, pin_brute_force, pin_split_combine, pin_cache_rows,
-            pin_normwise_rel_err, pin_out_projection, pin_kv_a_projection]
+            pin_normwise_rel_err, pin_out_projection, pin_kv_a_projection, pin_decompress_kv]

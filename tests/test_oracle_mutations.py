@@ -13,7 +13,7 @@ import pins
 ORIG = {name: getattr(om, name) for name in
         ["attention_naive", "attention_absorbed", "rope_angles", "rope", "rms_norm",
          "e4m3_encode", "combine_partials", "absorb_q", "out_uv", "round_to_bf16",
-          "normwise_rel_err", "out_projection", "kv_a_projection"]}
+          "normwise_rel_err", "out_projection", "kv_a_projection", "decompress_kv"]}
 
 
 def _patch(monkeypatch, name, fn):
@@ -139,10 +139,25 @@ def _kv_a_transposed_halves(monkeypatch):
     _patch(monkeypatch, "kv_a_projection", proj)
 
 
+def _decompress_swapped(monkeypatch):
+    def dec(c, w_uk, w_uv):
+        k, v = ORIG["decompress_kv"](c, w_uk, w_uv)
+        return v, k                                                  # keys from W_UV, values from W_UK
+    _patch(monkeypatch, "decompress_kv", dec)
+
+
+def _decompress_heads_reversed(monkeypatch):
+    def dec(c, w_uk, w_uv):
+        k, v = ORIG["decompress_kv"](c, w_uk, w_uv)
+        return k[:, ::-1], v[:, ::-1]                                # head i gets head H-1-i's weights
+    _patch(monkeypatch, "decompress_kv", dec)
+
+
 MUTATIONS = [_drop_rope_term, _scale_128, _rope_wrong_direction, _rope_half_split, _rms_no_sqrt,
              _causal_excludes_self, _e4m3_ties_away, _combine_no_weights, _wrong_value_matrix,
              _bf16_truncates, _gate_mean, _gate_den_from_got, _gate_wrong_axis, _gate_zero,
-             _gate_global_norm, _concat_interleaved, _kv_a_transposed_halves]
+             _gate_global_norm, _concat_interleaved, _kv_a_transposed_halves, _decompress_swapped,
+             _decompress_heads_reversed]
 
 
 @pytest.mark.parametrize("mutate", MUTATIONS, ids=lambda f: f.__name__.strip("_"))
