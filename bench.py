@@ -357,9 +357,10 @@ def run_gpu(args, w, rank, world, local_rank):
 
     # max over ranks
     elapsed_ms, e2e_ms, dec_ms = max_over_ranks([elapsed_ms, e2e_ms, float(np.mean(decode_ms))], world, dev)
-    extra = None
+    extra = level2 = None
     if world == 1 and not args.no_extra and w.name == "long":
         extra = time_extra(args, "fp8_mtp", dev, stream)
+        level2 = time_level2(args, dev, stream)
     if rank != 0:
         return 0
     tokens_per_step = w.batch * w.q_len
@@ -381,6 +382,8 @@ def run_gpu(args, w, rank, world, local_rank):
     }
     if extra is not None:
         line["fp8_mtp"] = extra
+    if level2 is not None:
+        line["level2_comparison"] = level2
     if not args.no_cpu_baseline and world == 1:
         v, reps, el, cores = time_oracle(w, heads=w.n_heads, budget_s=args.cpu_budget)
         line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
@@ -389,6 +392,60 @@ def run_gpu(args, w, rank, world, local_rank):
                                           f"cache built before timing"}
     print(json.dumps(line), flush=True)
     return 0
+
+
+def time_level2(args, dev, stream):
+    """The non-absorbed ("level 2") decode next to the absorbed one on the
+    one-sequence workload (v3_b1): per-head keys and values decompressed from
+    the latents (mla_decompress_kv) and standard attention over them
+    (mla_attend_naive), against absorb_q + decode + combine + out_uv, both
+    producing the per-head outputs.  Each timed after a 256 MB L2 flush."""
+    import torch
+    import latent_attention_decode_absorbed_b200 as mla
+    from workloads.device import DeviceWorkload
+    w = W.WORKLOADS["v3_b1"]
+    dw = DeviceWorkload(w, device=dev)
+    st = dw.step
+    H = w.n_heads
+    k_c = torch.empty((st.num_pages, 64, H, 128), dtype=torch.bfloat16, device=dev)
+    v_c = torch.empty_like(k_c)
+    out = torch.empty(st.out.shape, dtype=st.out.dtype, device=dev)
+    flush = torch.empty(int(256e6) // 4, dtype=torch.float32, device=dev)
+
+    def level2():
+        mla.mla_decompress_kv(st.cache, mla.MLA_BF16, st.num_pages, 64, dw.w_uk, dw.w_uv, H, k_c, v_c, st.err)
+        mla.mla_attend_naive(dw.q_nope, dw.q_pe, st.cache, mla.MLA_BF16, k_c, v_c, st.num_pages, st.block_table,
+                             st.max_pages, 64, st.seq_lens, w.batch, w.q_len, H, st.softmax_scale, out, None, st.err)
+
+    def absorbed():
+        st.absorb(dw.q_nope, dw.q_pe, dw.w_uk)
+        st.attend()
+        st.combine()
+        st.project_out(dw.w_uv)
+
+    res = {}
+    for name, fn in (("level2", level2), ("absorbed", absorbed)):
+        for _ in range(max(3, args.warmup)):
+            fn()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        for e in ev:
+            flush.fill_(1.0)
+            e[0].record(stream)
+            fn()
+            e[1].record(stream)
+        torch.cuda.synchronize()
+        res[name] = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    assert int(st.err.item()) == 0, "device error flag set"
+    kv_bytes = 2 * k_c.numel() * k_c.element_size()
+    line = {"config": workload_config(w, dw.lens), "steps": args.steps,
+            "level2_ms": res["level2"], "absorbed_ms": res["absorbed"],
+            "absorbed_speedup": res["level2"] / res["absorbed"],
+            "level2_kv_bytes": kv_bytes,
+            "note": "per-head outputs of one decode step; level2 = mla_decompress_kv + mla_attend_naive, "
+                    "absorbed = absorb_q + decode + combine + out_uv; CUDA events, L2 flushed before each"}
+    del dw, st, k_c, v_c, flush
+    torch.cuda.empty_cache()
+    return line
 
 
 def time_extra(args, name, dev, stream):
@@ -444,7 +501,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-extra", action="store_true", help="skip the e4m3 two-token line (long workload only)")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the e4m3 two-token line and the level-2 comparison (long workload only)")
     # smaller cases of a workload's shape, for profiler captures (not bench lines)
     ap.add_argument("--batch", type=int, default=None, help="override the workload's batch (profiling)")
     ap.add_argument("--seq-len", type=int, default=None, help="override the workload's fixed length (profiling)")

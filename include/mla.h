@@ -369,6 +369,45 @@ mla_status mla_decode_static(const void* q_abs, mla_dtype q_dtype, const void* c
                              void* o_lat, mla_dtype o_dtype, float* lse_out, int32_t* err_word,
                              cudaStream_t stream);
 
+/*
+ * The non-absorbed ("level 2") decode, for comparison with the path above
+ * ("HuggingFace version does NOT use efficient MLA caching", the ways MLA
+ * inference can be run: level 2 caches the latent and decompresses per-head
+ * keys and values at every step).  "DeepSeek-V2: MLA Explained", "MLA Full
+ * Formulas" parts 2 and 3.  bf16 caches with 64-row pages only.
+ *
+ * mla_decompress_kv
+ * For every row r of every page p of the pool (c = the row's 512 latent numbers):
+ *   k_c[p, r, h, :] = W_UK[h] c,   v_c[p, r, h, :] = W_UV[h] c      (fp32 sums, stored bf16)
+ *   cache       device bf16 [num_pages, 9, 64, 64] (the page-blocked pool), 128-byte aligned
+ *   w_uk, w_uv  device bf16 [n_heads, 128, 512] (as in mla_absorb_q / mla_out_uv)
+ *   k_c, v_c    device bf16 [num_pages, 64, n_heads, 128] each (num_pages * 64 * n_heads * 256 bytes)
+ *   err_word    device int32 or NULL (MLA_DEVERR_TIMEOUT if a bounded wait ran out)
+ * Errors: MLA_ERR_UNSUPPORTED for a cache that is not bf16 or page_size != 64.
+ */
+mla_status mla_decompress_kv(const void* cache, mla_dtype cache_dtype, int num_pages, int page_size,
+                             const void* w_uk, const void* w_uv, int n_heads, void* k_c, void* v_c,
+                             int32_t* err_word, cudaStream_t stream);
+
+/*
+ * mla_attend_naive
+ * Standard attention per head over the decompressed keys and values.  Query
+ * row r = b*q_len + t of sequence b sees the rows j <= seq_lens[b] - q_len + t
+ * (as in mla_decode_fwd); with k_j the row's rope key (cache columns 512..575):
+ *   z_j = softmax_scale * (q_nope[r,h,:] . k_c[j,h,:] + q_pe[r,h,:] . k_j)
+ *   out[r,h,:] = sum_j e^{z_j - m} v_c[j,h,:] / sum_j e^{z_j - m},   lse[r,h] = m + ln sum_j e^{z_j - m}
+ *   q_nope      device bf16 [batch*q_len, n_heads, 128];  q_pe  device bf16 [batch*q_len, n_heads, 64]
+ *   cache, k_c, v_c as produced for mla_decompress_kv; block_table, seq_lens as in mla_decode_fwd
+ *   out         device bf16 [batch*q_len, n_heads, 128];  lse  device float [batch*q_len, n_heads] or NULL
+ *   err_word    device int32 or NULL (MLA_DEVERR_PAGE for table entries outside the pool; those rows are skipped)
+ * out equals the absorbed path's mla_out_uv result up to rounding.
+ */
+mla_status mla_attend_naive(const void* q_nope, const void* q_pe, const void* cache, mla_dtype cache_dtype,
+                            const void* k_c, const void* v_c, int num_pages, const int32_t* block_table,
+                            int max_pages_per_seq, int page_size, const int32_t* seq_lens, int batch,
+                            int q_len, int n_heads, float softmax_scale, void* out, float* lse,
+                            int32_t* err_word, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

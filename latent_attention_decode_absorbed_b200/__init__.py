@@ -38,6 +38,8 @@ _SIGS = {
     "mla_out_proj": ("i", "pppiiip"),
     "mla_kv_proj_workspace_bytes": ("z", "i"),
     "mla_kv_proj_append": ("i", "ppiippppiiipfppippiipp"),
+    "mla_decompress_kv": ("i", "piiippipppp"),
+    "mla_attend_naive": ("i", "pppippipiipiiifpppp"),
 }
 _CT = {"p": ctypes.c_void_p, "i": ctypes.c_int, "f": ctypes.c_float, "d": ctypes.c_double,
        "s": ctypes.c_char_p, "z": ctypes.c_size_t, "Q": ctypes.c_ulonglong}
@@ -191,6 +193,26 @@ def mla_out_proj(out, w_o, u, rows, n_heads, d_model, stream=None):
     """u[r] = W_O [out[r, 0]; ...; out[r, H-1]] (fp32 u, overwritten)."""
     _check("mla_out_proj", lib().mla_out_proj(_ptr(out), _ptr(w_o), _ptr(u), int(rows), int(n_heads), int(d_model),
                                               _stream(stream)))
+
+
+def mla_decompress_kv(cache, cache_dtype, num_pages, page_size, w_uk, w_uv, n_heads, k_c, v_c, err_word=None,
+                      stream=None):
+    """Per-head keys and values of every cached row (the non-absorbed path's
+    decompression): k_c, v_c bf16 [num_pages, 64, n_heads, 128]."""
+    _check("mla_decompress_kv", lib().mla_decompress_kv(_ptr(cache), int(cache_dtype), int(num_pages), int(page_size),
+                                                        _ptr(w_uk), _ptr(w_uv), int(n_heads), _ptr(k_c), _ptr(v_c),
+                                                        _ptr(err_word), _stream(stream)))
+
+
+def mla_attend_naive(q_nope, q_pe, cache, cache_dtype, k_c, v_c, num_pages, block_table, max_pages_per_seq,
+                     page_size, seq_lens, batch, q_len, n_heads, softmax_scale, out, lse=None, err_word=None,
+                     stream=None):
+    """Standard attention per head over decompressed keys and values: out bf16
+    [batch*q_len, n_heads, 128], lse fp32 [batch*q_len, n_heads] (optional)."""
+    _check("mla_attend_naive", lib().mla_attend_naive(
+        _ptr(q_nope), _ptr(q_pe), _ptr(cache), int(cache_dtype), _ptr(k_c), _ptr(v_c), int(num_pages),
+        _ptr(block_table), int(max_pages_per_seq), int(page_size), _ptr(seq_lens), int(batch), int(q_len),
+        int(n_heads), float(softmax_scale), _ptr(out), _ptr(lse), _ptr(err_word), _stream(stream)))
 
 
 def mla_kv_proj_workspace_bytes(n_new) -> int:

@@ -186,6 +186,47 @@ mla_status mla_out_proj(const void* out, const void* w_o, float* u, int rows, in
   return cuda_status(launch_out_proj(out, w_o, u, rows, n_heads, d_model, stream), "mla_out_proj launch");
 }
 
+mla_status mla_decompress_kv(const void* cache, mla_dtype cache_dtype, int num_pages, int page_size,
+                             const void* w_uk, const void* w_uv, int n_heads, void* k_c, void* v_c, int32_t* err_word,
+                             cudaStream_t stream) {
+  MLA_REQUIRE(num_pages >= 0, MLA_ERR_INVALID_ARG, "mla_decompress_kv: num_pages < 0");
+  MLA_REQUIRE(cache_dtype == MLA_BF16, MLA_ERR_UNSUPPORTED, "mla_decompress_kv: the cache must be bf16");
+  MLA_REQUIRE(page_size == MLA_PAGE, MLA_ERR_UNSUPPORTED, "mla_decompress_kv: page_size must be %d", MLA_PAGE);
+  MLA_REQUIRE(n_heads >= 1 && n_heads <= MLA_MAX_HEADS, MLA_ERR_INVALID_ARG,
+              "mla_decompress_kv: n_heads must be in [1, %d]", MLA_MAX_HEADS);
+  MLA_REQUIRE(num_pages <= 2 * 65535, MLA_ERR_UNSUPPORTED, "mla_decompress_kv: more than %d pages", 2 * 65535);
+  if (num_pages == 0) return MLA_OK;
+  MLA_REQUIRE(cache && w_uk && w_uv && k_c && v_c, MLA_ERR_INVALID_ARG, "mla_decompress_kv: null pointer");
+  MLA_REQUIRE(aligned(cache, 128) && aligned(w_uk, 16) && aligned(w_uv, 16) && aligned(k_c, 16) && aligned(v_c, 16),
+              MLA_ERR_INVALID_ARG, "mla_decompress_kv: misaligned pointer");
+  return cuda_status(launch_decompress_kv(cache, num_pages, w_uk, w_uv, n_heads, k_c, v_c, err_word, stream),
+                     "mla_decompress_kv launch");
+}
+
+mla_status mla_attend_naive(const void* q_nope, const void* q_pe, const void* cache, mla_dtype cache_dtype,
+                            const void* k_c, const void* v_c, int num_pages, const int32_t* block_table,
+                            int max_pages_per_seq, int page_size, const int32_t* seq_lens, int batch, int q_len,
+                            int n_heads, float softmax_scale, void* out, float* lse, int32_t* err_word,
+                            cudaStream_t stream) {
+  MLA_REQUIRE(batch >= 0 && q_len >= 1 && num_pages >= 0 && max_pages_per_seq >= 1, MLA_ERR_INVALID_ARG,
+              "mla_attend_naive: bad sizes");
+  MLA_REQUIRE(cache_dtype == MLA_BF16, MLA_ERR_UNSUPPORTED, "mla_attend_naive: the cache must be bf16");
+  MLA_REQUIRE(page_size == MLA_PAGE, MLA_ERR_UNSUPPORTED, "mla_attend_naive: page_size must be %d", MLA_PAGE);
+  MLA_REQUIRE(n_heads >= 1 && n_heads <= MLA_MAX_HEADS, MLA_ERR_INVALID_ARG,
+              "mla_attend_naive: n_heads must be in [1, %d]", MLA_MAX_HEADS);
+  MLA_REQUIRE(softmax_scale > 0.f, MLA_ERR_INVALID_ARG, "mla_attend_naive: softmax_scale must be > 0");
+  MLA_REQUIRE((long long)batch * q_len <= 0x7fffffff, MLA_ERR_UNSUPPORTED, "mla_attend_naive: too many rows");
+  if (batch == 0) return MLA_OK;
+  MLA_REQUIRE(q_nope && q_pe && cache && k_c && v_c && block_table && seq_lens && out, MLA_ERR_INVALID_ARG,
+              "mla_attend_naive: null pointer");
+  MLA_REQUIRE(aligned(q_nope, 16) && aligned(q_pe, 16) && aligned(cache, 128) && aligned(k_c, 16) &&
+                  aligned(v_c, 16) && aligned(out, 16),
+              MLA_ERR_INVALID_ARG, "mla_attend_naive: misaligned pointer");
+  NaiveArgs a{q_nope, q_pe, cache, k_c, v_c, num_pages, block_table, max_pages_per_seq, seq_lens, batch, q_len,
+              n_heads, softmax_scale, out, lse, err_word};
+  return cuda_status(launch_attend_naive(a, stream), "mla_attend_naive launch");
+}
+
 size_t mla_kv_proj_workspace_bytes(int n_new) {
   if (n_new <= 0) return 0;
   return (size_t)n_new * MLA_D_ROW * sizeof(float) + (size_t)((n_new + 127) / 128) * sizeof(unsigned);

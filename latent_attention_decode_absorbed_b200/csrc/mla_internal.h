@@ -58,6 +58,17 @@ cudaError_t launch_out_proj(const void* out_heads, const void* w_o, float* u, in
 cudaError_t launch_kv_proj_append(const void* h, const void* w_kva, int d_model, float* workspace,
                                   const AppendArgs& a, cudaStream_t st);
 
+// the non-absorbed comparison path: per-head keys and values decompressed
+// from the latents, then standard attention per head
+cudaError_t launch_decompress_kv(const void* cache, int num_pages, const void* w_uk, const void* w_uv, int n_heads,
+                                 void* k_c, void* v_c, int32_t* err, cudaStream_t st);
+struct NaiveArgs {
+  const void* q_nope; const void* q_pe; const void* cache; const void* k_c; const void* v_c; int num_pages;
+  const int32_t* block_table; int max_pages; const int32_t* seq_lens; int batch; int q_len; int n_heads;
+  float softmax_scale; void* out; float* lse; int32_t* err;
+};
+cudaError_t launch_attend_naive(const NaiveArgs& a, cudaStream_t st);
+
 // shard_major: parts laid out [num_parts, rows, n_heads, 512] (per-GPU results
 // of a row-sharded sequence) instead of [rows, n_heads, num_parts, 512]
 cudaError_t launch_combine(const float* o_part, const float* lse_part, int rows, int n_heads,
