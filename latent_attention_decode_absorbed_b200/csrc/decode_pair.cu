@@ -782,7 +782,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<F8>::kThr
           const uint8_t* src = smem + kOffStg + ss * kStgBytes;
           uint8_t* dst = smem + kOffRing + slot * kSlotBytes;
           const int qq = lane & 3;
-#pragma unroll 4
+#pragma unroll
           for (int i = 0; i < 16; ++i) {
             const int box = i >> 3, row = (lane >> 2) + 8 * (i & 7);
             const uint4 codes = *reinterpret_cast<const uint4*>(src + box * kBox8 + row * 64 + qq * 16);
