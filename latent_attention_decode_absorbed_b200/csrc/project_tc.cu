@@ -55,7 +55,13 @@ struct Proj {
   static constexpr int KC = K / 64;                                  // 64-wide K chunks
   static constexpr int kABytes = KC * 128 * 128;                     // [128 rows x K] bf16
   static constexpr int kBBytes = K * NH * 2;
-  static constexpr int kSmem = kABytes + kBBytes + 1024 + 64;
+  // out_uv streams its eight K chunks (A [128 rows x 64] + B [64 N x 64]) through
+  // a four-stage ring: 96 KB instead of 192 KB, so two CTAs fit on an SM and the
+  // 256 CTAs of a 128-head step run in one wave; absorb_q (K = 128) loads at once
+  static constexpr int kStages = KIND == 0 ? 1 : 4;
+  static constexpr int kStageA = 128 * 128, kStageB = NH * 128, kStage = kStageA + kStageB;
+  static constexpr int kOperands = KIND == 0 ? kABytes + kBBytes : kStages * kStage;
+  static constexpr int kSmem = kOperands + 1024 + 128;
   static constexpr uint32_t kTmemCols = NH < 32 ? 32 : NH;
 };
 
@@ -68,14 +74,19 @@ __global__ void __launch_bounds__(kPThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t s_a = smem_u32(smem), s_b = s_a + P::kABytes;
-  uint8_t* misc = smem + P::kABytes + P::kBBytes;
-  const uint32_t bar_full = smem_u32(misc), bar_done = bar_full + 8, tslot = bar_full + 16;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 20);
+  uint8_t* misc = smem + P::kOperands;
+  // barriers: full[kStages], empty[kStages], done; then the TMEM slot and the abort flag
+  const uint32_t bar_full = smem_u32(misc), bar_empty = bar_full + 8 * P::kStages,
+                 bar_done = bar_full + 16 * P::kStages, tslot = bar_done + 8;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 16 * P::kStages + 12);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.x, m0 = blockIdx.y * 128, nh = blockIdx.z;
 
   if (threadIdx.x == 0) {
-    mbar_init(bar_full, 1);
+    for (int i = 0; i < P::kStages; ++i) {
+      mbar_init(bar_full + 8 * i, 1);
+      mbar_init(bar_empty + 8 * i, 1);
+    }
     mbar_init(bar_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -84,35 +95,26 @@ __global__ void __launch_bounds__(kPThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(misc + 16);
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(misc + 16 * P::kStages + 8);
 
   bool ok = true;
-  if (threadIdx.x == 0) {
+  if (threadIdx.x == 0 && KIND == 0) {
     mbar_arrive_expect_tx(bar_full, P::kABytes + P::kBBytes);
     for (int c = 0; c < P::KC; ++c)   // rows m0.., K chunk c: [128 rows x 64] (rows past the end read as 0)
       tma_load_3d(s_a + c * 128 * 128, &tm_a, 64 * c, h, m0, bar_full);
-    if (KIND == 0) {
-      // W_UK[h] as [128 K rows x 64 N] boxes, N-major: 4 blocks of 64 N
-      for (int nb = 0; nb < P::NH / 64; ++nb)
-        tma_load_3d(s_b + nb * (P::K * 128), &tm_b, P::NH * nh + 64 * nb, 0, h, bar_full);
-    } else {
-      // W_UV[h] rows (N) nh*64.., K chunk c: [64 N rows x 64 K], K-major
-      for (int c = 0; c < P::KC; ++c)
-        tma_load_3d(s_b + c * (P::NH * 128), &tm_b, 64 * c, P::NH * nh, h, bar_full);
-    }
+    // W_UK[h] as [128 K rows x 64 N] boxes, N-major: 4 blocks of 64 N
+    for (int nb = 0; nb < P::NH / 64; ++nb)
+      tma_load_3d(s_b + nb * (P::K * 128), &tm_b, P::NH * nh + 64 * nb, 0, h, bar_full);
     ok = mbar_wait<false>(bar_full, 0, abort_flag);
     if (ok) {
       tc_fence_after();
-      constexpr uint32_t idesc = idesc_f16(128, P::NH, false, KIND == 0);
+      constexpr uint32_t idesc = idesc_f16(128, P::NH, false, true);
       for (int c = 0; c < P::KC; ++c) {
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
           const uint64_t ad = smem_desc_sw128(s_a + c * 128 * 128 + ks * 32, 16, 1024);
-          uint64_t bd;
-          if (KIND == 0)   // N-major: 8 K rows per 1 KB atom, 64-N blocks kK*128 bytes apart
-            bd = smem_desc_sw128(s_b + (4 * c + ks) * 2048, P::K * 128, 1024);
-          else             // K-major: like A
-            bd = smem_desc_sw128(s_b + c * (P::NH * 128) + ks * 32, 16, 1024);
+          // N-major: 8 K rows per 1 KB atom, 64-N blocks kK*128 bytes apart
+          const uint64_t bd = smem_desc_sw128(s_b + (4 * c + ks) * 2048, P::K * 128, 1024);
           mma_f16_cta(tmem, ad, bd, idesc, (c | ks) != 0);
         }
       }
@@ -120,6 +122,38 @@ __global__ void __launch_bounds__(kPThreads, 1)
     } else {
       *abort_flag = 1;
     }
+  } else if (threadIdx.x == 0) {
+    // out_uv: stage c holds rows m0.. of K chunk c ([128 x 64], rows past the end read as 0)
+    // and W_UV[h] rows (N) nh*64.. of K chunk c ([64 x 64], K-major)
+    auto load = [&](int c) {
+      const int slot = c % P::kStages;
+      const uint32_t dst = s_a + slot * P::kStage;
+      mbar_arrive_expect_tx(bar_full + 8 * slot, P::kStage);
+      tma_load_3d(dst, &tm_a, 64 * c, h, m0, bar_full + 8 * slot);
+      tma_load_3d(dst + P::kStageA, &tm_b, 64 * c, P::NH * nh, h, bar_full + 8 * slot);
+    };
+    for (int c = 0; c < P::kStages && c < P::KC; ++c) load(c);
+    constexpr uint32_t idesc = idesc_f16(128, P::NH, false, false);
+    for (int c = 0; c < P::KC && ok; ++c) {
+      const int slot = c % P::kStages;
+      const uint32_t ph = (c / P::kStages) & 1u;
+      ok = mbar_wait<false>(bar_full + 8 * slot, ph, abort_flag);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t a0 = s_a + slot * P::kStage;
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks)
+        mma_f16_cta(tmem, smem_desc_sw128(a0 + ks * 32, 16, 1024),
+                    smem_desc_sw128(a0 + P::kStageA + ks * 32, 16, 1024), idesc, (c | ks) != 0);
+      mma_commit_cta(bar_empty + 8 * slot);
+      if (c + P::kStages < P::KC) {
+        // the slot is reused once these MMAs have read it
+        ok = mbar_wait<false>(bar_empty + 8 * slot, ph, abort_flag);
+        if (ok) load(c + P::kStages);
+      }
+    }
+    if (ok) mma_commit_cta(bar_done);
+    else *abort_flag = 1;
   }
   __syncthreads();
   if (!*abort_flag) ok = __all_sync(0xffffffffu, mbar_wait<false>(bar_done, 0, abort_flag));
