@@ -16,7 +16,8 @@ import math
 import numpy as np
 
 from . import (D_C, D_R, D_ROW, D_V, MLA_BF16, MLA_E4M3, MLA_F32, PAGE, mla_absorb_q, mla_cache_append,
-               mla_combine, mla_decode_fwd, mla_out_uv, mla_rope_table)
+               mla_combine, mla_decode_fwd, mla_kv_proj_append, mla_kv_proj_workspace_bytes, mla_out_proj,
+               mla_out_uv, mla_rope_table)
 
 _DT = {"f32": MLA_F32, "bf16": MLA_BF16, "e4m3": MLA_E4M3}
 
@@ -95,6 +96,30 @@ class DecodeStep:
 
     def project_out(self, w_uv, stream=None):
         mla_out_uv(self.o_lat, w_uv, self.out, self.batch * self.q_len, self.n_heads, self.dtype, stream)
+
+    # -- the projections on either side of the path ---------------------------
+    def append_from_hidden(self, h, w_kva, seq_ids, positions, stream=None):
+        """The new tokens' cache rows straight from hidden states h (bf16
+        [n_new, d_model]): kv_a = h W_kv,a^T, then the rows of mla_cache_append,
+        in one launch (mla_kv_proj_append).  w_kva: bf16 [576, d_model]."""
+        n_new, d_model = int(h.shape[0]), int(h.shape[1])
+        need = mla_kv_proj_workspace_bytes(n_new)
+        ws = getattr(self, "_kv_ws", None)
+        if ws is None or ws.numel() < need:
+            ws = self._kv_ws = self.torch.empty((max(need, 1),), dtype=self.torch.uint8, device=self.device)
+        mla_kv_proj_append(h, w_kva, n_new, d_model, ws, seq_ids, positions, self.block_table, self.batch,
+                           self.max_pages, PAGE, self.norm_gain, self.eps, self.rope_cos, self.rope_sin,
+                           self.max_pos, self.cache, self.cache_scale, self.cache_dtype, self.num_pages, self.err,
+                           stream)
+
+    def project_model(self, w_o, u=None, stream=None):
+        """u = W_O [out_1; ...; out_H] for every query row (mla_out_proj on the
+        step's `out`); w_o: bf16 [d_model, H*128]; returns u, fp32 [rows, d_model]."""
+        rows, d_model = self.batch * self.q_len, int(w_o.shape[0])
+        if u is None:
+            u = self.torch.empty((rows, d_model), dtype=self.torch.float32, device=self.device)
+        mla_out_proj(self.out, w_o, u, rows, self.n_heads, d_model, stream)
+        return u
 
     # -- the whole step ----------------------------------------------------
     def run(self, kv_a_new, seq_ids, positions, q_nope, q_pe, w_uk, w_uv, stream=None):

@@ -134,3 +134,48 @@ def test_kv_proj_append_matches_oracle(cache_dt, lens):
                                                             eps), cache_dt)[0]
     stored = oracle.stored_rows(ref, cache_dt)[0]
     assert oracle.normwise_rel_err(stored[:, None, :], full[:, None, :]) < {"f32": 1e-5, "bf16": 1e-2, "e4m3": 3e-2}[cache_dt]
+
+
+@pytest.mark.parametrize("cache_dt", ["bf16", "e4m3"])
+def test_layer_chain_from_hidden_states(cache_dt):
+    """One layer end to end through DecodeStep: the step's new tokens enter as
+    hidden states (append_from_hidden: W_kv,a, then the cache rows), attention
+    over the whole cache, W_UV per head, then W_O over all heads
+    (project_model); against the oracle's fp64 chain on the same inputs."""
+    import workloads as W
+    from gpu_common import TOL
+    from workloads.device import DeviceWorkload
+    w = W.Workload("chain_" + cache_dt, 3, 2, 128, None, (130, 400), "bf16", cache_dt, True, 256, seed=21)
+    dw = DeviceWorkload(w)            # the cache holds the workload's rows at every position
+    st = dw.step
+    g = np.random.default_rng(77)
+    n = w.batch * w.q_len
+    h = round_bf16(g.standard_normal((n, D_MODEL)).astype(np.float32))
+    w_kva = round_bf16((g.standard_normal((576, D_MODEL)) / np.sqrt(D_MODEL)).astype(np.float32))
+    w_o = round_bf16((g.standard_normal((D_MODEL, w.n_heads * 128)) / np.sqrt(w.n_heads * 128)).astype(np.float32))
+    # the new tokens (the last q_len positions of each sequence) come from h
+    st.append_from_hidden(to_device(h, "bf16"), to_device(w_kva, "bf16"), dw.seq_ids, dw.positions)
+    st.absorb(dw.q_nope, dw.q_pe, dw.w_uk)
+    st.attend()
+    st.combine()
+    st.project_out(dw.w_uv)
+    u = st.project_model(to_device(w_o, "bf16"))
+    torch.cuda.synchronize()
+    assert int(st.err.item()) == 0
+    got = to_host_f64(u).reshape(w.batch, w.q_len, D_MODEL)
+    qn, qp = W.queries(w)
+    wuk, wuv = W.weights(w)
+    sid, pos = dw.seq_ids.cpu().numpy(), dw.positions.cpu().numpy()
+    for b, L in enumerate(dw.lens):
+        L = int(L)
+        old = oracle.sequence_cache(W.kv_rows(w, b)[:L - w.q_len], cache_dt, None, w.eps, w.theta)
+        mine = np.flatnonzero(sid == b)
+        mine = mine[np.argsort(pos[mine])]
+        new = oracle.stored_rows(oracle.cache_rows_from_hidden(h[mine].astype(np.float64), w_kva.astype(np.float64),
+                                                               pos[mine], None, w.eps, w.theta), cache_dt)[0]
+        c_hat = np.concatenate([old[0], new[:, :512]])
+        k_r = np.concatenate([old[1], new[:, 512:]])
+        rows = slice(b * w.q_len, (b + 1) * w.q_len)
+        out = oracle.attention_absorbed(qn[rows], qp[rows], wuk, wuv, c_hat, k_r)[0]
+        ref = oracle.out_projection(out, w_o.astype(np.float64))
+        assert oracle.normwise_rel_err(got[b][:, None, :], ref[:, None, :]) < TOL[cache_dt], f"seq {b}"
