@@ -14,6 +14,8 @@ namespace {
 
 template <typename IN, int CK>  // CK: MLA_F32, MLA_BF16, MLA_E4M3
 __global__ void __launch_bounds__(256) append_kernel(AppendArgs a) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= a.n_new) return;
@@ -31,11 +33,10 @@ cudaError_t launch_in(const AppendArgs& a, cudaStream_t st) {
   dim3 block(256);
   dim3 grid((a.n_new + 7) / 8);
   switch (a.cache_dtype) {
-    case MLA_F32: append_kernel<IN, MLA_F32><<<grid, block, 0, st>>>(a); break;
-    case MLA_BF16: append_kernel<IN, MLA_BF16><<<grid, block, 0, st>>>(a); break;
-    default: append_kernel<IN, MLA_E4M3><<<grid, block, 0, st>>>(a); break;
+    case MLA_F32: return launch_dependent(append_kernel<IN, MLA_F32>, grid, block, 0, st, a);
+    case MLA_BF16: return launch_dependent(append_kernel<IN, MLA_BF16>, grid, block, 0, st, a);
+    default: return launch_dependent(append_kernel<IN, MLA_E4M3>, grid, block, 0, st, a);
   }
-  return cudaGetLastError();
 }
 
 }  // namespace

@@ -27,6 +27,8 @@ __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ 
                                                       OT* __restrict__ o_lat, float* __restrict__ lse_out) {
   extern __shared__ float w[];               // [S] weights
   __shared__ float red[4];
+  griddep_wait();
+  griddep_launch_dependents();
   const size_t rh = blockIdx.x;
   const float* lp = lse_part + rh * st.l_rh;
   // max over splits
@@ -86,11 +88,10 @@ cudaError_t launch_combine(const float* o_part, const float* lse_part, int rows,
   const PartStrides ps = shard_major ? PartStrides{n * MLA_D_C, MLA_D_C, n, 1}
                                      : PartStrides{MLA_D_C, (size_t)num_parts * MLA_D_C, 1, (size_t)num_parts};
   if (o_dtype == MLA_F32)
-    combine_kernel<float><<<(unsigned)n, 128, smem, st>>>(o_part, lse_part, num_parts, ps, (float*)o_lat, lse_out);
-  else
-    combine_kernel<__nv_bfloat16><<<(unsigned)n, 128, smem, st>>>(o_part, lse_part, num_parts, ps,
-                                                                  (__nv_bfloat16*)o_lat, lse_out);
-  return cudaGetLastError();
+    return launch_dependent(combine_kernel<float>, dim3((unsigned)n), dim3(128), smem, st, o_part, lse_part,
+                            num_parts, ps, (float*)o_lat, lse_out);
+  return launch_dependent(combine_kernel<__nv_bfloat16>, dim3((unsigned)n), dim3(128), smem, st, o_part, lse_part,
+                          num_parts, ps, (__nv_bfloat16*)o_lat, lse_out);
 }
 
 }  // namespace mla

@@ -230,10 +230,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<F8>::kThr
   };
 
   // ---- set-up
-  // the pair's first unit is claimed now, so that the counter's round trip
-  // overlaps the barrier and tensor-memory set-up
-  unsigned first_claim = 0;
-  if (leader && threadIdx.x == 0) first_claim = atomicAdd(p.claim, 1u);
   if (threadIdx.x == 0) {
     for (int i = 0; i < kSlots; ++i) {
       mbar_init(bar(kBFull + i), F8 ? 2 : 1);
@@ -265,6 +261,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<F8>::kThr
   cluster_sync();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(misc + kMTmem);
+  // the set-up above may overlap the previous kernel on the stream; global
+  // memory (the unit counter included) only after it has completed.  The
+  // pair's first unit is claimed at once, so that the counter's round trip
+  // overlaps the rest of the start.
+  griddep_wait();
+  griddep_launch_dependents();
+  unsigned first_claim = 0;
+  if (leader && threadIdx.x == 0) first_claim = atomicAdd(p.claim, 1u);
 
   // ---- the pair's unit sequence: the leader's producer claims units from the
   // launch's counter and posts them, in order, to a queue in both CTAs
@@ -966,10 +970,10 @@ cudaError_t launch_decode_pair(const DecodeArgs& a, cudaStream_t st) {
   if (!claim_slot(a.o_part, &p.claim, &p.done)) return cudaErrorInvalidSymbol;
   const long long pairs = units < P ? units : P;
   if (f8)
-    decode_pair_kernel<true><<<dim3((unsigned)(2 * pairs)), PairLayout<true>::kThreads, smem, st>>>(tc, tc2, tq, p);
-  else
-    decode_pair_kernel<false><<<dim3((unsigned)(2 * pairs)), PairLayout<false>::kThreads, smem, st>>>(tc, tc2, tq, p);
-  return cudaGetLastError();
+    return launch_dependent(decode_pair_kernel<true>, dim3((unsigned)(2 * pairs)), dim3(PairLayout<true>::kThreads),
+                            smem, st, tc, tc2, tq, p);
+  return launch_dependent(decode_pair_kernel<false>, dim3((unsigned)(2 * pairs)), dim3(PairLayout<false>::kThreads),
+                          smem, st, tc, tc2, tq, p);
 }
 
 }  // namespace mla

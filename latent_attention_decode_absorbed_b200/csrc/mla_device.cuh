@@ -11,6 +11,16 @@
 
 namespace mla {
 
+// Programmatic dependent launch.  griddep_wait: wait until the kernel before
+// this one on the stream has completed and its memory is visible (returns at
+// once when this launch did not allow an early start).  Everything before it
+// may overlap the previous kernel, so it touches no global memory.
+// griddep_launch_dependents: the next kernel may begin its own set-up.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

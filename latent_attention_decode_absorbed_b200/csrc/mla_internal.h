@@ -75,6 +75,26 @@ cudaError_t launch_combine(const float* o_part, const float* lse_part, int rows,
                            int num_parts, bool shard_major, void* o_lat, int o_dtype, float* lse_out,
                            cudaStream_t st);
 
+// Launches `kernel` with programmatic dependent launch allowed: it may start
+// (its set-up, up to griddep_wait()) while the previous kernel on the stream
+// is still running.  Used for the kernels of the decode step, which all call
+// griddep_wait() before touching global memory.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                             Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // Bound (SM cycles, about 2 s at 2 GHz) of every barrier wait in the
 // tensor-core decode kernels, and the test hook that withholds one query load
 // (both set through mla_test_set_decode_wait, read at launch).

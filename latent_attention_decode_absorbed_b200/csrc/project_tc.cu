@@ -96,6 +96,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(misc + 16 * P::kStages + 8);
+  griddep_wait();
+  griddep_launch_dependents();
 
   bool ok = true;
   if (threadIdx.x == 0 && KIND == 0) {
@@ -233,9 +235,8 @@ cudaError_t launch_kind(const CUtensorMap& ta, const CUtensorMap& tb, const void
   cudaError_t e = cudaFuncSetAttribute(proj_tc_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize, P::kSmem);
   if (e != cudaSuccess) return e;
   dim3 grid(H, (rows + 127) / 128, 2);
-  proj_tc_kernel<KIND><<<grid, kPThreads, P::kSmem, st>>>(ta, tb, static_cast<const __nv_bfloat16*>(q_pe),
-                                                          static_cast<__nv_bfloat16*>(out), rows, H, err);
-  return cudaGetLastError();
+  return launch_dependent(proj_tc_kernel<KIND>, grid, dim3(kPThreads), P::kSmem, st, ta, tb,
+                          static_cast<const __nv_bfloat16*>(q_pe), static_cast<__nv_bfloat16*>(out), rows, H, err);
 }
 
 }  // namespace
