@@ -136,7 +136,7 @@ class DecodeStep:
     # -- the step as CUDA graphs ------------------------------------------------
     def capture(self, kv_a_new, seq_ids, positions, q_nope, q_pe, w_uk, w_uv, host_in=(), host_out=None):
         """Record the step's five calls as three CUDA graphs on this device:
-        `pre` (append, absorb), `attend` (the split-KV decode) and `post`
+        `pre` (append and absorb, as parallel branches), `attend` (the split-KV decode) and `post`
         (combine, out_uv).  A replay launches the same kernels with the same
         arguments; the graphs read the given tensors and write `out` in place,
         so the caller refreshes the inputs' contents before each replay.
@@ -150,10 +150,18 @@ class DecodeStep:
             for dst, src in host_in:
                 dst.copy_(src, non_blocking=True)
 
+        # append and absorb_q are independent: in the graph they are two
+        # branches (append on a forked stream), joined before the attention
+        fork = torch.cuda.Stream(device=self.device)
+
         def pre():
             copies_in()
-            self.append(kv_a_new, seq_ids, positions)
+            main = torch.cuda.current_stream(self.device)
+            fork.wait_stream(main)
+            with torch.cuda.stream(fork):
+                self.append(kv_a_new, seq_ids, positions)
             self.absorb(q_nope, q_pe, w_uk)
+            main.wait_stream(fork)
 
         def post():
             self.combine()
