@@ -377,7 +377,7 @@ def run_gpu(args, w, rank, world, local_rank):
         "roofline": roofline,
         "decode": _decode_summary(alg_bytes, alg_flops, dec_ms, elapsed_ms / args.steps, pk),
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": step.LAUNCHES_PER_STEP * args.steps,
+        "gpu_launches": step.launches_per_step * args.steps,
         "clocks": clocks,
     }
     if extra is not None:
@@ -420,8 +420,7 @@ def time_level2(args, dev, stream):
     def absorbed():
         st.absorb(dw.q_nope, dw.q_pe, dw.w_uk)
         st.attend()
-        st.combine()
-        st.project_out(dw.w_uv)
+        st.finish(dw.w_uv)
 
     res = {}
     for name, fn in (("level2", level2), ("absorbed", absorbed)):
@@ -442,7 +441,7 @@ def time_level2(args, dev, stream):
             "absorbed_speedup": res["level2"] / res["absorbed"],
             "level2_kv_bytes": kv_bytes,
             "note": "per-head outputs of one decode step; level2 = mla_decompress_kv + mla_attend_naive, "
-                    "absorbed = absorb_q + decode + combine + out_uv; CUDA events, L2 flushed before each"}
+                    "absorbed = absorb_q + decode + combine + out_uv (one launch for the last two at this size); CUDA events, L2 flushed before each"}
     del dw, st, k_c, v_c, flush
     torch.cuda.empty_cache()
     return line

@@ -267,6 +267,22 @@ mla_status mla_combine_shards(const float* o_shard, const float* lse_shard, int 
                               cudaStream_t stream);
 
 /*
+ * mla_combine_out_uv
+ * mla_combine followed by mla_out_uv in one launch, for bf16 and few query
+ * rows (each CTA reads one head's whole W_UV, so it suits steps of up to a few
+ * rows; the projection itself is "MLA Full Formulas" part 2 applied after the
+ * attention sum, as in mla_out_uv):
+ *   o_lat[r,h,:] as mla_combine (stored bf16, rounded as mla_combine rounds it; o_lat may be NULL)
+ *   out[r,h,:] = W_UV[h] o_lat[r,h,:]   (the bf16 o_lat, fp32 sums, stored bf16)
+ *   o_part, lse_part as for mla_combine;  w_uv device bf16 [n_heads, 128, 512]
+ *   o_lat device bf16 [rows, n_heads, 512] or NULL;  out device bf16 [rows, n_heads, 128]
+ *   lse_out device float [rows, n_heads] or NULL
+ */
+mla_status mla_combine_out_uv(const float* o_part, const float* lse_part, int rows, int n_heads,
+                              int num_splits, const void* w_uv, void* o_lat, void* out, float* lse_out,
+                              cudaStream_t stream);
+
+/*
  * mla_out_uv
  * Value up-projection applied after the softmax sum ("DeepSeek-V2: MLA
  * Explained", "MLA Full Formulas" part 2, v^C = W^UV c, moved past the sum per

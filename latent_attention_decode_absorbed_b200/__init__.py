@@ -39,6 +39,7 @@ _SIGS = {
     "mla_kv_proj_workspace_bytes": ("z", "i"),
     "mla_kv_proj_append": ("i", "ppiippppiiipfppippiipp"),
     "mla_decompress_kv": ("i", "piiippipppp"),
+    "mla_combine_out_uv": ("i", "ppiiippppp"),
     "mla_attend_naive": ("i", "pppippipiipiiifpppp"),
 }
 _CT = {"p": ctypes.c_void_p, "i": ctypes.c_int, "f": ctypes.c_float, "d": ctypes.c_double,
@@ -193,6 +194,13 @@ def mla_out_proj(out, w_o, u, rows, n_heads, d_model, stream=None):
     """u[r] = W_O [out[r, 0]; ...; out[r, H-1]] (fp32 u, overwritten)."""
     _check("mla_out_proj", lib().mla_out_proj(_ptr(out), _ptr(w_o), _ptr(u), int(rows), int(n_heads), int(d_model),
                                               _stream(stream)))
+
+
+def mla_combine_out_uv(o_part, lse_part, rows, n_heads, num_splits, w_uv, o_lat, out, lse_out=None, stream=None):
+    """mla_combine then mla_out_uv in one launch (bf16, few rows); o_lat may be None."""
+    _check("mla_combine_out_uv", lib().mla_combine_out_uv(_ptr(o_part), _ptr(lse_part), int(rows), int(n_heads),
+                                                          int(num_splits), _ptr(w_uv), _ptr(o_lat), _ptr(out),
+                                                          _ptr(lse_out), _stream(stream)))
 
 
 def mla_decompress_kv(cache, cache_dtype, num_pages, page_size, w_uk, w_uv, n_heads, k_c, v_c, err_word=None,

@@ -279,6 +279,20 @@ mla_status mla_combine(const float* o_part, const float* lse_part, int rows, int
                      "mla_combine launch");
 }
 
+mla_status mla_combine_out_uv(const float* o_part, const float* lse_part, int rows, int n_heads, int num_splits,
+                              const void* w_uv, void* o_lat, void* out, float* lse_out, cudaStream_t stream) {
+  MLA_REQUIRE(rows >= 0 && n_heads >= 1 && n_heads <= MLA_MAX_HEADS && num_splits >= 1, MLA_ERR_INVALID_ARG,
+              "mla_combine_out_uv: need rows >= 0, n_heads in [1, %d], num_splits >= 1", MLA_MAX_HEADS);
+  MLA_REQUIRE(num_splits <= 8192, MLA_ERR_UNSUPPORTED, "mla_combine_out_uv: num_splits above 8192");
+  if (rows == 0) return MLA_OK;
+  MLA_REQUIRE(o_part && lse_part && w_uv && out, MLA_ERR_INVALID_ARG, "mla_combine_out_uv: null pointer");
+  MLA_REQUIRE(aligned(o_part, 16) && aligned(w_uv, 16) && aligned(out, 16) && (!o_lat || aligned(o_lat, 16)),
+              MLA_ERR_INVALID_ARG, "mla_combine_out_uv: pointers must be 16-byte aligned");
+  return cuda_status(launch_combine_out_uv(o_part, lse_part, rows, n_heads, num_splits, w_uv, o_lat, out, lse_out,
+                                           stream),
+                     "mla_combine_out_uv launch");
+}
+
 mla_status mla_combine_shards(const float* o_shard, const float* lse_shard, int num_shards, int rows,
                               int n_heads, void* o_lat, mla_dtype o_dtype, float* lse_out, cudaStream_t stream) {
   MLA_REQUIRE(rows >= 0 && n_heads >= 1 && n_heads <= MLA_MAX_HEADS && num_shards >= 1, MLA_ERR_INVALID_ARG,

@@ -69,6 +69,10 @@ struct NaiveArgs {
 };
 cudaError_t launch_attend_naive(const NaiveArgs& a, cudaStream_t st);
 
+// the merge and the value up-projection in one launch (bf16, few query rows)
+cudaError_t launch_combine_out_uv(const float* o_part, const float* lse_part, int rows, int n_heads, int num_splits,
+                                  const void* w_uv, void* o_lat, void* out, float* lse_out, cudaStream_t st);
+
 // shard_major: parts laid out [num_parts, rows, n_heads, 512] (per-GPU results
 // of a row-sharded sequence) instead of [rows, n_heads, num_parts, 512]
 cudaError_t launch_combine(const float* o_part, const float* lse_part, int rows, int n_heads,

@@ -16,7 +16,7 @@ import math
 import numpy as np
 
 from . import (D_C, D_R, D_ROW, D_V, MLA_BF16, MLA_E4M3, MLA_F32, PAGE, mla_absorb_q, mla_cache_append,
-               mla_combine, mla_decode_fwd, mla_kv_proj_append, mla_kv_proj_workspace_bytes, mla_out_proj,
+               mla_combine, mla_combine_out_uv, mla_decode_fwd, mla_kv_proj_append, mla_kv_proj_workspace_bytes, mla_out_proj,
                mla_out_uv, mla_rope_table)
 
 _DT = {"f32": MLA_F32, "bf16": MLA_BF16, "e4m3": MLA_E4M3}
@@ -97,6 +97,27 @@ class DecodeStep:
     def project_out(self, w_uv, stream=None):
         mla_out_uv(self.o_lat, w_uv, self.out, self.batch * self.q_len, self.n_heads, self.dtype, stream)
 
+    # bf16 steps of at most this many query rows merge the splits and apply W_UV
+    # in one launch (mla_combine_out_uv); larger ones use the tensor-core GEMM
+    FUSED_POST_ROWS = 8
+
+    @property
+    def fused_post(self):
+        return self.dtype == MLA_BF16 and self.batch * self.q_len <= self.FUSED_POST_ROWS
+
+    def finish(self, w_uv, stream=None):
+        """After the attention: o_lat, lse and out (combine, then out_uv)."""
+        if self.fused_post:
+            mla_combine_out_uv(self.o_part, self.lse_part, self.batch * self.q_len, self.n_heads, self.num_splits,
+                               w_uv, self.o_lat, self.out, self.lse, stream)
+        else:
+            self.combine(stream)
+            self.project_out(w_uv, stream)
+
+    @property
+    def launches_per_step(self):
+        return 4 if self.fused_post else 5
+
     # -- the projections on either side of the path ---------------------------
     def append_from_hidden(self, h, w_kva, seq_ids, positions, stream=None):
         """The new tokens' cache rows straight from hidden states h (bf16
@@ -127,11 +148,9 @@ class DecodeStep:
         self.append(kv_a_new, seq_ids, positions, stream)
         self.absorb(q_nope, q_pe, w_uk, stream)
         self.attend(stream)
-        self.combine(stream)
-        self.project_out(w_uv, stream)
+        self.finish(w_uv, stream)
         return self.out
 
-    LAUNCHES_PER_STEP = 5
 
     # -- the step as CUDA graphs ------------------------------------------------
     def capture(self, kv_a_new, seq_ids, positions, q_nope, q_pe, w_uk, w_uv, host_in=(), host_out=None):
@@ -164,8 +183,7 @@ class DecodeStep:
             main.wait_stream(fork)
 
         def post():
-            self.combine()
-            self.project_out(w_uv)
+            self.finish(w_uv)
             if host_out is not None:
                 host_out.copy_(self.out, non_blocking=True)
 

@@ -180,6 +180,43 @@ def test_combine(S, dt):
     assert np.all(np.isneginf(got_l[~fin])) and np.all(got_o[~fin] == 0)
 
 
+@pytest.mark.parametrize("rows,H,S", [(1, 128, 32), (3, 16, 7), (8, 128, 1), (2, 65, 64)])
+def test_combine_out_uv(rows, H, S):
+    """The merge and W_UV in one launch: o_lat bit-identical to mla_combine,
+    out against the oracle (out_uv of the merged partials) and the two-launch
+    path."""
+    g = np.random.default_rng(rows * 100 + S)
+    o = g.standard_normal((rows, H, S, 512)).astype(np.float32)
+    lse = (g.standard_normal((rows, H, S)) * 3).astype(np.float32)
+    if S > 1:
+        lse[:, :, 1] = -np.inf                               # an empty split
+    lse[0, 0, :] = -np.inf                                   # a head that saw nothing
+    if S == 1:
+        lse[0, 0, 0] = 2.0
+    w_uv = round_bf16((g.standard_normal((H, 128, 512)) / np.sqrt(512)).astype(np.float32))
+    od, ld, wd = torch.from_numpy(o).cuda(), torch.from_numpy(lse).cuda(), to_device(w_uv, "bf16")
+    o_lat = torch.full((rows, H, 512), float("nan"), dtype=torch.bfloat16, device="cuda")
+    out = torch.full((rows, H, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse_out = torch.empty((rows, H), dtype=torch.float32, device="cuda")
+    mla.mla_combine_out_uv(od, ld, rows, H, S, wd, o_lat, out, lse_out)
+    o_lat2 = torch.empty_like(o_lat)
+    out2 = torch.empty_like(out)
+    lse2 = torch.empty_like(lse_out)
+    mla.mla_combine(od, ld, rows, H, S, o_lat2, mla.MLA_BF16, lse2)
+    mla.mla_out_uv(o_lat2, wd, out2, rows, H, mla.MLA_BF16)
+    torch.cuda.synchronize()
+    assert torch.equal(o_lat, o_lat2) and torch.equal(lse_out, lse2)
+    ref_o, _ = oracle.combine_partials(o, lse)
+    ref_out = oracle.out_uv(oracle.round_to_bf16(np.nan_to_num(ref_o)), w_uv.astype(np.float64))
+    got = to_host_f64(out)
+    assert np.all(np.isfinite(got))
+    seen = np.isfinite(lse).any(axis=2)                      # (row, head) pairs with a visible row
+    assert np.all(got[~seen] == 0)
+    assert oracle.normwise_rel_err(got[seen][:, None, :], ref_out[seen][:, None, :]) < 4e-3
+    # the same products as the tensor-core out_uv up to fp32 summation order and one bf16 rounding
+    np.testing.assert_allclose(got, to_host_f64(out2), rtol=2 ** -7, atol=1e-3)
+
+
 # ------------------------------------------------------------------ attention partials
 def _random_cache(g, num_pages, cache_dt):
     """Seeded cache contents straight from the generator: a valid input to the
