@@ -97,13 +97,16 @@ class DecodeStep:
     def project_out(self, w_uv, stream=None):
         mla_out_uv(self.o_lat, w_uv, self.out, self.batch * self.q_len, self.n_heads, self.dtype, stream)
 
-    # bf16 steps of at most this many query rows merge the splits and apply W_UV
-    # in one launch (mla_combine_out_uv); larger ones use the tensor-core GEMM
-    FUSED_POST_ROWS = 8
-
     @property
     def fused_post(self):
-        return self.dtype == MLA_BF16 and self.batch * self.q_len <= self.FUSED_POST_ROWS
+        """bf16 steps whose (query row, head) pairs fit in one wave of CTAs, one
+        per SM (each stages a head's 128 KB W_UV), merge the splits and apply
+        W_UV in one launch (mla_combine_out_uv); larger ones use combine and the
+        tensor-core GEMM (8 rows x 128 heads fused: a 33 us longer step)."""
+        if self.dtype != MLA_BF16:
+            return False
+        sms = self.torch.cuda.get_device_properties(self.device).multi_processor_count
+        return self.batch * self.q_len * self.n_heads <= sms
 
     def finish(self, w_uv, stream=None):
         """After the attention: o_lat, lse and out (combine, then out_uv)."""
@@ -154,9 +157,10 @@ class DecodeStep:
 
     # -- the step as CUDA graphs ------------------------------------------------
     def capture(self, kv_a_new, seq_ids, positions, q_nope, q_pe, w_uk, w_uv, host_in=(), host_out=None):
-        """Record the step's five calls as three CUDA graphs on this device:
-        `pre` (append and absorb, as parallel branches), `attend` (the split-KV decode) and `post`
-        (combine, out_uv).  A replay launches the same kernels with the same
+        """Record the step's calls as CUDA graphs on this device: `pre` (append
+        and absorb, as parallel branches), `attend` (the split-KV decode), `post`
+        (combine and out_uv, or their fused form) and `whole` (all of them in
+        one graph).  A replay launches the same kernels with the same
         arguments; the graphs read the given tensors and write `out` in place,
         so the caller refreshes the inputs' contents before each replay.
 
@@ -198,7 +202,7 @@ class DecodeStep:
         torch.cuda.current_stream(self.device).wait_stream(side)
         torch.cuda.synchronize(self.device)
         graphs = []
-        for fn in parts:
+        for fn in parts + (lambda: [f() for f in parts],):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, capture_error_mode="thread_local"):
                 fn()
@@ -207,13 +211,12 @@ class DecodeStep:
 
 
 class StepGraphs:
-    """The three graphs of one captured step; `replay()` runs them in order
-    on the current stream."""
+    """The graphs of one captured step: `pre`, `attend` and `post` (for timing
+    the attention between them) and `whole`, the same launches as one graph,
+    which `replay()` runs on the current stream."""
 
-    def __init__(self, pre, attend, post):
-        self.pre, self.attend, self.post = pre, attend, post
+    def __init__(self, pre, attend, post, whole):
+        self.pre, self.attend, self.post, self.whole = pre, attend, post, whole
 
     def replay(self):
-        self.pre.replay()
-        self.attend.replay()
-        self.post.replay()
+        self.whole.replay()
