@@ -86,7 +86,8 @@ constexpr int kMAbort = kMTmem + 4;
 constexpr int kMRedMax = kMTmem + 16;     // float [2 tile parities][2 lane halves][2 column halves][64 heads]
 constexpr int kMRedSum = kMRedMax + 2 * 4 * kHPC * 4;   // float [2 lane halves][2 column halves][64 heads]
 constexpr int kMUnitQ = kMRedSum + 4 * kHPC * 4;
-constexpr int kMiscBytes = kMUnitQ + 4 * kQN;
+constexpr int kMStgSeq = kMUnitQ + 4 * kQN;   // int [8]: e4m3, the stage each staging slot was last filled for
+constexpr int kMiscBytes = kMStgSeq + 4 * 8;
 
 // Shared memory, barriers and threads of the bf16 (F8 = false) and e4m3
 // (F8 = true) kernels.  With an e4m3 cache the producer's copies land in a
@@ -123,7 +124,17 @@ struct PairLayout {
   static constexpr int kBEnd = kBQReady + 1;
   static_assert(kSmem <= 227 * 1024, "shared memory budget");
   static_assert(kBEnd <= 48, "barrier area");
+  static_assert(kStg <= 8, "staging sequence area");
 };
+
+__device__ __forceinline__ int ld_acquire_shared(const int* p) {
+  int v;
+  asm volatile("ld.acquire.cta.shared::cta.b32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_shared(int* p, int v) {
+  asm volatile("st.release.cta.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
 
 struct PairParams {
   int n_heads, q_len, batch;
@@ -240,6 +251,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<F8>::kThr
       mbar_init(bar(kBStgEmpty + i), 1);
     }
     if (F8) mbar_init(bar(kBQReady), 2 * kConvWarps);
+    for (int i = 0; i < kStg; ++i) reinterpret_cast<int*>(misc + kMStgSeq)[i] = -1;
     mbar_init(bar(kBSFull), 1);
     mbar_init(bar(kBSFull + 1), 1);
     mbar_init(bar(kBODone), 1);
@@ -368,6 +380,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<F8>::kThr
             const uint32_t ph = (kc / kStg) & 1u;
             if (!mbar_wait<false>(bar(kBStgEmpty + slot), ph ^ 1u, abort_flag, lim)) return false;
             mbar_arrive_expect_tx(bar(kBStgFull + slot), kStgBytes);
+            // the converter of this stage checks this before its parity wait (see there)
+            st_release_shared(reinterpret_cast<int*>(misc + kMStgSeq) + slot, (int)kc);
             dst = s_base + kOffStg + slot * kStgBytes;
             fb = bar(kBStgFull + slot);
           } else {
@@ -780,6 +794,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<F8>::kThr
           if (scale_page >= 0) {
             s_lo = __ldg(p.cache_scale + (size_t)scale_page * 64 + lane);
             s_hi = __ldg(p.cache_scale + (size_t)scale_page * 64 + 32 + lane);
+          }
+          // Staging slots are shared by the converter warps (stage my uses slot
+          // my % kStg, warp my % kConvWarps), so this warp may get here while the
+          // slot's previous fill (stage my - kStg, another warp's) is still
+          // pending; a parity wait would then match the phase before that and
+          // pass early.  The producer records each fill's stage once the slot is
+          // free again, which is after its previous phase completed: wait for that.
+          {
+            const int* seq = reinterpret_cast<const int*>(misc + kMStgSeq) + ss;
+            const uint64_t t0 = clock64();
+            bool okw = true;
+            for (uint32_t n = 1; ld_acquire_shared(seq) != (int)my; ++n) {
+              if ((n & 255u) == 0 && (*abort_flag || clock64() - t0 > lim)) {
+                *abort_flag = 1;
+                okw = false;
+                break;
+              }
+            }
+            if (!__all_sync(0xffffffffu, okw)) return false;
           }
           if (!__all_sync(0xffffffffu, mbar_wait<false>(bar(kBStgFull + ss), sph, abort_flag, lim))) return false;
           if (!__all_sync(0xffffffffu, mbar_wait<false>(bar(kBEmpty + slot), ph ^ 1u, abort_flag, lim))) return false;
