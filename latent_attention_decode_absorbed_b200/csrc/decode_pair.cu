@@ -1,5 +1,8 @@
-// Split-KV latent attention for 65..128 heads over a bf16 cache, on the
-// tcgen05 tensor cores, with the heads split between the two CTAs of a pair.
+// Split-KV latent attention for 65..128 heads over a bf16 or e4m3 cache, on
+// the tcgen05 tensor cores, with the heads split between the two CTAs of a
+// pair.  With an e4m3 cache (the F8 instantiation) converter warps widen the
+// staged codes into the same f16 operand layout, Q and P are f16, and the
+// softmax applies each row's dequantisation scale to its scores.
 //
 // What it computes ("DeepSeek-V2: MLA Explained", "MLA Full Formulas" part 3
 // with the absorption of "Optimization Note"): for each head h of query row
@@ -30,6 +33,7 @@
 // half, lanes 64-127: the upper 128).
 //
 // Cache rows stream through a ring of seven 16 KB shared-memory stages
+// (e4m3: four, widened from six 8 KB staging slots of raw codes)
 // filled by TMA (128-byte swizzle) in the order the MMA consumes them: per
 // tile the nine score stages of tile i+1 follow the value stages of tile i,
 // so the score GEMM runs a tile ahead of the value GEMM and the softmax of a
