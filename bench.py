@@ -50,15 +50,24 @@ def peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
-def binding_roofline(alg_bytes, alg_flops, launch_ms, pk, traffic):
+def tensor_peak(pk, mma):
+    """Dense tensor peak for the decode's MMA operand type: the measured bf16
+    figure (also the f16 one), or for e4m3 operands that figure times the
+    nominal dense ratio 2 (4.5 against 2.25 PFLOP/s)."""
+    return pk["bf16_tflops"] * (2.0 if mma == "e4m3" else 1.0)
+
+
+def binding_roofline(alg_bytes, alg_flops, launch_ms, pk, traffic, mma="bf16"):
     """The decode launch against its binding roofline: the cache bytes at the
-    HBM peak or the contraction FLOPs at the bf16 tensor peak (also the f16
-    peak the e4m3 cache's widened operands run at), whichever takes longer."""
+    HBM peak or the contraction FLOPs at the tensor peak of its MMA operand
+    type (bf16; f16 for the widened e4m3 cache; e4m3 for the 8-bit form),
+    whichever takes longer."""
     s = launch_ms / 1e3
-    if alg_flops / (pk["bf16_tflops"] * 1e12) > alg_bytes / (pk["hbm_gbs"] * 1e9):
+    tpk = tensor_peak(pk, mma)
+    if alg_flops / (tpk * 1e12) > alg_bytes / (pk["hbm_gbs"] * 1e9):
         achieved = alg_flops / s / 1e12
-        r = {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-             "frac": achieved / pk["bf16_tflops"], "traffic": traffic}
+        r = {"bound": "tensor", "achieved": achieved, "peak": tpk, "unit": "TFLOP/s",
+             "frac": achieved / tpk, "traffic": traffic, "mma": mma}
     else:
         achieved = alg_bytes / s / 1e9
         r = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
@@ -66,6 +75,13 @@ def binding_roofline(alg_bytes, alg_flops, launch_ms, pk, traffic):
     r.update({"kernel": "mla_decode_fwd", "peak_source": pk["source"], "algorithmic_bytes_per_launch": alg_bytes,
               "algorithmic_flops_per_launch": alg_flops, "launch_ms": launch_ms})
     return r
+
+
+def mma_type(step):
+    """Operand type of the decode's MMAs for a DecodeStep."""
+    if getattr(step, "q8", False):
+        return "e4m3"
+    return "f16" if step.cache_dtype == 2 else "bf16"
 
 
 def decode_src_hash():
@@ -283,10 +299,11 @@ def _timed_steps(torch, step_fn, steps, stream, flush, barrier, decode_events=Tr
     return total, [e[0].elapsed_time(e[1]) for e in dec] if decode_events else []
 
 
-def _decode_summary(alg_bytes, alg_flops, dec_ms, step_ms, pk):
-    roof_ms = 1e3 * max(alg_bytes / (pk["hbm_gbs"] * 1e9), alg_flops / (pk["bf16_tflops"] * 1e12))
+def _decode_summary(alg_bytes, alg_flops, dec_ms, step_ms, pk, mma="bf16"):
+    tpk = tensor_peak(pk, mma)
+    roof_ms = 1e3 * max(alg_bytes / (pk["hbm_gbs"] * 1e9), alg_flops / (tpk * 1e12))
     return {"cache_gbs": alg_bytes / (dec_ms / 1e3) / 1e9, "tflops": alg_flops / (dec_ms / 1e3) / 1e12,
-            "tensor_frac_burst": alg_flops / (dec_ms / 1e3) / 1e12 / pk["bf16_tflops"],
+            "tensor_frac_burst": alg_flops / (dec_ms / 1e3) / 1e12 / tpk,
             "roofline_ms": roof_ms, "roofline_frac": roof_ms / dec_ms, "share_of_step": dec_ms / step_ms}
 
 
@@ -368,14 +385,14 @@ def run_gpu(args, w, rank, world, local_rank):
     e2e_value = job_throughput(world, tokens_per_step, args.steps, e2e_ms)
     pk = peaks()
     traffic = recorded_traffic(w.name)
-    roofline = binding_roofline(alg_bytes, alg_flops, dec_ms, pk, traffic)
+    roofline = binding_roofline(alg_bytes, alg_flops, dec_ms, pk, traffic, mma_type(step))
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
         "data": "synthetic", "config": workload_config(w, lens),
         "roofline": roofline,
-        "decode": _decode_summary(alg_bytes, alg_flops, dec_ms, elapsed_ms / args.steps, pk),
+        "decode": _decode_summary(alg_bytes, alg_flops, dec_ms, elapsed_ms / args.steps, pk, mma_type(step)),
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": step.launches_per_step * args.steps,
         "clocks": clocks,
@@ -483,8 +500,8 @@ def time_extra(args, name, dev, stream):
     out = {"config": workload_config(w, dw.lens), "steps": args.steps,
            "value": w.batch * w.q_len * args.steps / (total_ms / 1e3), "unit": "tokens/s",
            "ms_per_step": total_ms / args.steps,
-           "roofline": binding_roofline(alg_bytes, alg_flops, dec_ms, pk, recorded_traffic(name)),
-           "decode": _decode_summary(alg_bytes, alg_flops, dec_ms, total_ms / args.steps, pk),
+           "roofline": binding_roofline(alg_bytes, alg_flops, dec_ms, pk, recorded_traffic(name), mma_type(step)),
+           "decode": _decode_summary(alg_bytes, alg_flops, dec_ms, total_ms / args.steps, pk, mma_type(step)),
            "clocks": clk.summary()}
     del graphs, dw, step
     torch.cuda.empty_cache()

@@ -233,6 +233,52 @@ mla_status mla_decode_fwd(const void* q_abs, mla_dtype q_dtype, const void* cach
                           cudaStream_t stream);
 
 /*
+ * mla_split_q_e4m3
+ * The two-term e4m3 form of bf16 absorbed queries: the query operand of
+ * mla_decode_fwd_q8.  Not a step of the method itself: with an e4m3 cache
+ * ("DeepSeek'in MLA'si latent attention ile KV cache'i %93 sikistiriyor",
+ * cache section; OCP FP8 E4M3) both GEMMs of the decode can run on 8-bit
+ * tensor-core MMAs, whose two operands are both 8-bit, and one e4m3 rounding
+ * of the query (relative 2^-4) would move the scores too far.  Per (row r,
+ * head h), in fp32 round-to-nearest-even:
+ *   a = max|q_abs[r,h,:]|, inv = 448 / a (0 when a = 0), y = q_abs * inv
+ *   q8[r, 0, h, :] = e4m3(y)              (hi; saturating)
+ *   q8[r, 1, h, :] = e4m3(y - hi)         (lo; y - hi is exact)
+ *   q_scale[r, h]  = a / 448
+ * so that q_abs ~ q_scale * (hi + lo) to about 2^-8 relative.
+ *   q_abs   device bf16 [rows, n_heads, 576]  (16-byte aligned)
+ *   q8      device uint8 [rows, 2, n_heads, 576] e4m3 codes (16-byte aligned), caller-owned
+ *   q_scale device float [rows, n_heads], caller-owned
+ * rows >= 0 (0 is a no-op), 1 <= n_heads <= 128.
+ */
+mla_status mla_split_q_e4m3(const void* q_abs, int rows, int n_heads, void* q8, float* q_scale,
+                            cudaStream_t stream);
+
+/*
+ * mla_decode_fwd_q8
+ * mla_decode_fwd over an E4M3 cache with both GEMMs on 8-bit tensor-core
+ * MMAs (tcgen05 kind::f8f6f4), for 65..128 heads: the same outputs and
+ * conventions (o_part, lse_part, merged runs of splits, pool contract,
+ * concurrency rule) with the query given in the two-term form of
+ * mla_split_q_e4m3.  The scores are q_scale[r,h] * cache_scale[j] * the code
+ * GEMM of (hi + lo) with row j's codes; the value GEMM's weights are carried
+ * as two e4m3 terms too, with each row's scale folded in relative to the
+ * largest scale among the rows of the unit of work, so that o_part holds
+ *   sum_j e^{z_j - m} (codes_j * cache_scale[j])[0:512] / sum_j e^{z_j - m}
+ * to within about 2^-8 relative per weight.  The running maximum m is
+ * raised once a tile's scores exceed it by 4 (log2 units), which keeps each
+ * weight below 448.
+ *   q8, q_scale  from mla_split_q_e4m3 for batch*q_len rows and n_heads
+ *   other arguments as for mla_decode_fwd with cache_dtype E4M3
+ * Supported: page_size 64, 65 <= n_heads <= 128 (else MLA_ERR_UNSUPPORTED).
+ */
+mla_status mla_decode_fwd_q8(const void* q8, const float* q_scale, const void* cache, const float* cache_scale,
+                             int num_pages, const int32_t* block_table, int max_pages_per_seq, int page_size,
+                             const int32_t* seq_lens, int batch, int q_len, int n_heads, int num_splits,
+                             int split_tokens, float softmax_scale, float* o_part, float* lse_part,
+                             int32_t* err_word, cudaStream_t stream);
+
+/*
  * mla_combine
  * Log-sum-exp merge of split partials (the softmax sum of "MLA Full Formulas"
  * part 3 decomposed over disjoint row ranges):

@@ -30,6 +30,8 @@ _SIGS = {
     "mla_cache_append": ("i", "piipppiiipfppippiipp"),
     "mla_absorb_q": ("i", "ppppiiip"),
     "mla_decode_fwd": ("i", "pippiipiipiiiiifpppp"),
+    "mla_split_q_e4m3": ("i", "piippp"),
+    "mla_decode_fwd_q8": ("i", "ppppipiipiiiiifpppp"),
     "mla_combine": ("i", "ppiiipipp"),
     "mla_combine_shards": ("i", "ppiiipipp"),
     "mla_out_uv": ("i", "pppiiip"),
@@ -155,6 +157,23 @@ def mla_decode_fwd(q_abs, q_dtype, cache, cache_scale, cache_dtype, num_pages, b
         _ptr(block_table), int(max_pages_per_seq), int(page_size), _ptr(seq_lens), int(batch),
         int(q_len), int(n_heads), int(num_splits), int(split_tokens), float(softmax_scale),
         _ptr(o_part), _ptr(lse_part), _ptr(err_word), _stream(stream)))
+
+
+def mla_split_q_e4m3(q_abs, rows, n_heads, q8, q_scale, stream=None):
+    """bf16 q_abs [rows, H, 576] -> two-term e4m3 q8 [rows, 2, H, 576] (uint8) and q_scale [rows, H]."""
+    _check("mla_split_q_e4m3", lib().mla_split_q_e4m3(_ptr(q_abs), int(rows), int(n_heads), _ptr(q8), _ptr(q_scale),
+                                                      _stream(stream)))
+
+
+def mla_decode_fwd_q8(q8, q_scale, cache, cache_scale, num_pages, block_table, max_pages_per_seq, page_size,
+                      seq_lens, batch, q_len, n_heads, num_splits, split_tokens, softmax_scale, o_part, lse_part,
+                      err_word=None, stream=None):
+    """mla_decode_fwd over an e4m3 cache on 8-bit MMAs, from mla_split_q_e4m3's query form."""
+    _check("mla_decode_fwd_q8", lib().mla_decode_fwd_q8(
+        _ptr(q8), _ptr(q_scale), _ptr(cache), _ptr(cache_scale), int(num_pages), _ptr(block_table),
+        int(max_pages_per_seq), int(page_size), _ptr(seq_lens), int(batch), int(q_len), int(n_heads),
+        int(num_splits), int(split_tokens), float(softmax_scale), _ptr(o_part), _ptr(lse_part), _ptr(err_word),
+        _stream(stream)))
 
 
 def mla_combine(o_part, lse_part, rows, n_heads, num_splits, o_lat, o_dtype, lse_out=None, stream=None):

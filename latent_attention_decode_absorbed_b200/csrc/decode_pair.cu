@@ -73,39 +73,48 @@ constexpr int kSlotBytes = 16384;         // one stage: one score chunk or one v
 constexpr int kBox = 8192;                // [64 rows x 64 16-bit values]
 constexpr int kBox8 = 4096;               // e4m3 cache: [64 rows x 64 codes]
 constexpr int kStgBytes = 2 * kBox8;      // e4m3 cache: the raw codes of one stage
+constexpr int kSlot8 = 2 * kBox8;         // 8-bit MMAs: one stage of codes ([128 rows x 64] or [64 rows x 128])
+constexpr int kQ8Plane = kChunks * kBox8; // 8-bit MMAs: one term (hi or lo) of Q, 9 x [64 heads x 64 codes]
 constexpr int kQChunk = kHPC * 128;       // [64 heads x 64 dims], 16-bit
 constexpr int kPChunk = kHPC * 128;       // [64 heads x 64 rows], 16-bit: P of one page
 constexpr int kWarpProd = 0, kWarpMma = 1, kWarpSoft0 = 2, kSoftWarps = 8;
 constexpr int kWarpConv0 = kWarpSoft0 + kSoftWarps, kConvWarps = 4;   // e4m3 cache: converters
 constexpr int kQN = 8;                    // unit queue depth
 constexpr float kRescaleLog2 = 8.0f;      // lazy rescale threshold (log2 units)
+constexpr float kRescaleLog2Q8 = 4.0f;    // 8-bit MMAs: probabilities stay <= 2^4, and times
+constexpr float kPScale8 = 16.0f;         // 16 x (row scale / segment's largest) <= 256 < 448
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;             // S of tile t at kColS + 128 (t & 1)
 constexpr uint32_t kColO = 256;           // O: dims 0..255 at 256, dims 256..511 at 384
 
 // offsets inside the misc area
-constexpr int kMBars = 0;                 // 48 barriers
-constexpr int kMTmem = 48 * 8;
+constexpr int kMBars = 0;                 // 64 barriers
+constexpr int kMTmem = 64 * 8;
 constexpr int kMAbort = kMTmem + 4;
 constexpr int kMRedMax = kMTmem + 16;     // float [2 tile parities][2 lane halves][2 column halves][64 heads]
 constexpr int kMRedSum = kMRedMax + 2 * 4 * kHPC * 4;   // float [2 lane halves][2 column halves][64 heads]
 constexpr int kMUnitQ = kMRedSum + 4 * kHPC * 4;
 constexpr int kMStgSeq = kMUnitQ + 4 * kQN;   // int [8]: e4m3, the stage each staging slot was last filled for
-constexpr int kMiscBytes = kMStgSeq + 4 * 8;
+constexpr int kMScMax = kMStgSeq + 4 * 8;     // float [2 segment parities][8 softmax warps]: 8-bit MMAs
+constexpr int kMiscBytes = kMScMax + 4 * 2 * kSoftWarps;
 
-// Shared memory, barriers and threads of the bf16 (F8 = false) and e4m3
-// (F8 = true) kernels.  With an e4m3 cache the producer's copies land in a
-// staging ring of raw codes and four converter warps widen them into the
-// operand ring (one slot fewer, to make room for the staging).
-template <bool F8>
+// Shared memory, barriers and threads of the bf16 (F8 = D8 = false), the
+// widening e4m3 (F8) and the 8-bit MMA e4m3 (D8) kernels.  With F8 the
+// producer's copies land in a staging ring of raw codes and four converter
+// warps widen them into the operand ring (one slot fewer, to make room for
+// the staging).  With D8 the codes are the operands: stages are half the
+// size, so the ring has twice the stages.
+template <bool F8, bool D8 = false>
 struct PairLayout {
-  static constexpr int kSlots = F8 ? kConvWarps : 7;      // operand ring stages (e4m3: one per converter)
+  static_assert(!(F8 && D8), "one e4m3 form at a time");
+  static constexpr int kSlotB = D8 ? kSlot8 : kSlotBytes;  // bytes of one operand stage
+  static constexpr int kSlots = F8 ? kConvWarps : (D8 ? 14 : 7);   // operand ring stages
   static constexpr int kStg = F8 ? 6 : 0;                 // staging slots
   static constexpr int kThreads = 32 * (kWarpSoft0 + kSoftWarps + (F8 ? kConvWarps : 0));
   // bytes from the 1024-aligned base
-  static constexpr int kOffQ = 0;                          // Q: 9 x 8 KB, K-major SW128
+  static constexpr int kOffQ = 0;                          // Q: 9 x 8 KB, K-major SW128 (D8: hi, lo 9 x 4 KB, SW64)
   static constexpr int kOffRing = kOffQ + kChunks * kQChunk;
-  static constexpr int kOffP = kOffRing + kSlots * kSlotBytes;   // P: 4 pages x 8 KB, K-major SW128
+  static constexpr int kOffP = kOffRing + kSlots * kSlotB;   // P: 4 pages x 8 KB (D8: hi, lo 4 KB each)
   static constexpr int kOffStg = kOffP + 4 * kPChunk;
   static constexpr int kOffMisc = kOffStg + kStg * kStgBytes;
   static constexpr int kSmem = kOffMisc + kMiscBytes + 1024;     // + alignment slack
@@ -127,7 +136,7 @@ struct PairLayout {
   static constexpr int kBQReady = kBStgEmpty + kStg;    // leader: both CTAs' Q widened to f16
   static constexpr int kBEnd = kBQReady + 1;
   static_assert(kSmem <= 227 * 1024, "shared memory budget");
-  static_assert(kBEnd <= 48, "barrier area");
+  static_assert(kBEnd <= 64, "barrier area");
   static_assert(kStg <= 8, "staging sequence area");
 };
 
@@ -156,6 +165,7 @@ struct PairParams {
   unsigned long long wait_limit;
   int withhold_q;
   const float* cache_scale;    // e4m3 cache: per-row dequantisation scale [num_pages * 64]
+  const float* q_scale;        // 8-bit MMAs: per (query row, head) scale of the two-term query [rows * n_heads]
 };
 
 // page id of a cached row of sequence b (0 for rows outside the table or the
@@ -183,11 +193,11 @@ __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
 
 // tm_cache: boxes of one [64 rows x 64 columns] block (e4m3: [64 x 64 codes]);
 // tm_cache2: boxes of two adjacent blocks (bf16 only); tm_q: q_abs boxes.
-template <bool F8>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<F8>::kThreads, 1)
+template <bool F8, bool D8 = false>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<F8, D8>::kThreads, 1)
     decode_pair_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_constant__ CUtensorMap tm_cache2,
                        const __grid_constant__ CUtensorMap tm_q, const PairParams p) {
-  using L = PairLayout<F8>;
+  using L = PairLayout<F8, D8>;
   constexpr int kSlots = L::kSlots, kStg = L::kStg;
   constexpr int kOffQ = L::kOffQ, kOffRing = L::kOffRing, kOffP = L::kOffP, kOffStg = L::kOffStg,
                 kOffMisc = L::kOffMisc;
@@ -358,6 +368,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<F8>::kThr
             mbar_arrive_expect_tx(bar(kBQFull), kChunks * kQChunk);
             for (int c = 0; c < kChunks; ++c)
               tma_load_3d(s_q + c * kQChunk, &tm_q, 64 * c, (int)rank * kHPC, r, bar(kBQFull));
+          } else if constexpr (D8) {
+            // both terms of the query (planes 2r and 2r + 1 of the map), 64-byte swizzled
+            const uint32_t q_bar = mapa(bar(kBQFull), 0);
+            if (leader) mbar_arrive_expect_tx(bar(kBQFull), 2u * 2u * kQ8Plane);
+            for (int hl = 0; hl < 2; ++hl)
+              for (int c = 0; c < kChunks; ++c)
+                tma_load_3d_pair(s_q + hl * kQ8Plane + c * kBox8, &tm_q, 64 * c, (int)rank * kHPC, 2 * r + hl, q_bar);
           } else {
             const uint32_t q_bar = mapa(bar(kBQFull), 0);
             if (leader) mbar_arrive_expect_tx(bar(kBQFull), 2u * kChunks * kQChunk);
@@ -392,8 +409,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<F8>::kThr
             const uint32_t slot = kc % kSlots;
             const uint32_t ph = (kc / kSlots) & 1u;
             if (!mbar_wait<false>(bar(kBEmpty + slot), ph ^ 1u, abort_flag, lim)) return false;
-            if (leader) mbar_arrive_expect_tx(bar(kBFull + slot), 2u * kSlotBytes);
-            dst = s_ring + slot * kSlotBytes;
+            if (leader) mbar_arrive_expect_tx(bar(kBFull + slot), 2u * L::kSlotB);
+            dst = s_ring + slot * L::kSlotB;
             fb = mapa(bar(kBFull + slot), 0);
           }
           ++kc;
@@ -409,7 +426,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<F8>::kThr
               tma_load_2d_hint(dst + kBox8, &tm_cache, 0, (pg1 * kChunks + c) * 64, fb, pol_keep);
             } else {
               tma_load_2d_pair_hint(dst, &tm_cache, 0, (pg0 * kChunks + c) * 64, fb, pol_keep);
-              tma_load_2d_pair_hint(dst + kBox, &tm_cache, 0, (pg1 * kChunks + c) * 64, fb, pol_keep);
+              tma_load_2d_pair_hint(dst + (D8 ? kBox8 : kBox), &tm_cache, 0, (pg1 * kChunks + c) * 64, fb, pol_keep);
             }
           }
           return true;
@@ -470,15 +487,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<F8>::kThr
     // O(i-1) is done (one P buffer), so running the score GEMM further ahead
     // only delays O(i) (measured slower).
     if (leader) {
-      // e4m3 cache: the operands are f16 (widened codes, Q and P in f16)
-      constexpr uint32_t idS = idesc_f16(128, 256, false, false, F8);
-      constexpr uint32_t idO = idesc_f16(128, 256, false, true, F8);
+      // F8: the operands are f16 (widened codes, Q and P in f16); D8: e4m3
+      constexpr uint32_t idS = D8 ? idesc_e4m3(128, 256, false, false) : idesc_f16(128, 256, false, false, F8);
+      constexpr uint32_t idO = D8 ? idesc_e4m3(128, 256, false, true) : idesc_f16(128, 256, false, true, F8);
       auto ready = [&](uint32_t& src, uint32_t& empty) -> bool {
         const uint32_t slot = kc % kSlots;
         const uint32_t ph = (kc / kSlots) & 1u;
         if (!__all_sync(0xffffffffu, mbar_wait<false>(bar(kBFull + slot), ph, abort_flag, lim))) return false;
         tc_fence_after();
-        src = s_ring + slot * kSlotBytes;
+        src = s_ring + slot * L::kSlotB;
         empty = bar(kBEmpty + slot);
         ++kc;
         return true;
@@ -502,14 +519,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<F8>::kThr
           const uint32_t t = gt + i;
           const uint32_t sb = t & 1u;
           const uint32_t d = tmem + kColS + 128 * sb;
-          const uint64_t qd = smem_desc_sw128(s_q, 16, 1024);
           for (int c = 0; c < kChunks; ++c) {
             uint32_t a0, empty;
             if (!ready(a0, empty)) return false;
-            const uint64_t kd = smem_desc_sw128(a0, 16, 1024);
+            if constexpr (D8) {
+              // K = 32 codes per MMA (+32 bytes along the 64-byte lines), both
+              // query terms into the same accumulator
+              const uint64_t qd = smem_desc_sw64(s_q, 16, 512);
+              const uint64_t kd = smem_desc_sw64(a0, 16, 512);
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks)   // K = 16 per MMA: +32 bytes along the 128-byte lines
-              mma_pair_f16_w(d, qd + ((c * kQChunk + ks * 32) >> 4), kd + ((ks * 32) >> 4), idS, (c | ks) != 0);
+              for (int ks = 0; ks < 2; ++ks)
+#pragma unroll
+                for (int hl = 0; hl < 2; ++hl)
+                  mma_pair_e4m3_w(d, qd + ((hl * kQ8Plane + c * kBox8 + ks * 32) >> 4), kd + ((ks * 32) >> 4), idS,
+                                  (c | ks | hl) != 0);
+            } else {
+              const uint64_t qd = smem_desc_sw128(s_q, 16, 1024);
+              const uint64_t kd = smem_desc_sw128(a0, 16, 1024);
+#pragma unroll
+              for (int ks = 0; ks < 4; ++ks)   // K = 16 per MMA: +32 bytes along the 128-byte lines
+                mma_pair_f16_w(d, qd + ((c * kQChunk + ks * 32) >> 4), kd + ((ks * 32) >> 4), idS, (c | ks) != 0);
+            }
             mma_commit_pair_w(empty, 0x3);
           }
           mma_commit_pair_w(bar(kBSFull + sb), 0x3);
@@ -526,17 +556,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<F8>::kThr
               !__all_sync(0xffffffffu, mbar_wait(bar(kBEpiDone), (uc - 1) & 1, abort_flag, lim)))
             return false;
           tc_fence_after();
-          const uint64_t pd = smem_desc_sw128(s_p, 16, 1024);
           for (int pg_i = 0; pg_i < 4; ++pg_i) {
             if (lo + kTile * j + 64 * pg_i >= hi) break;
             for (int bb = 0; bb < 2; ++bb) {
               uint32_t b0, empty;
               if (!ready(b0, empty)) return false;
-              const uint64_t vd = smem_desc_sw128(b0, kBox, 1024);
+              if constexpr (D8) {
+                // 32 rows per MMA: +32 bytes of the P lines, +2 KB of V (8-row
+                // groups of 512 bytes); the stage's two 64-dim blocks 4 KB apart;
+                // both probability terms into the same accumulator
+                const uint64_t pd = smem_desc_sw64(s_p, 16, 512);
+                const uint64_t vd = smem_desc_sw64(b0, kBox8, 512);
 #pragma unroll
-              for (int ks = 0; ks < 4; ++ks)   // 16 rows per MMA: +32 bytes of P lines, +2 KB of V lines
-                mma_pair_f16_w(tmem + kColO + 128 * bb, pd + ((pg_i * kPChunk + ks * 32) >> 4),
-                               vd + ((ks * 2048) >> 4), idO, (j | pg_i | ks) != 0);
+                for (int ks = 0; ks < 2; ++ks)
+#pragma unroll
+                  for (int hl = 0; hl < 2; ++hl)
+                    mma_pair_e4m3_w(tmem + kColO + 128 * bb, pd + ((pg_i * kPChunk + hl * kBox8 + ks * 32) >> 4),
+                                    vd + ((ks * 2048) >> 4), idO, (j | pg_i | ks | hl) != 0);
+              } else {
+                const uint64_t pd = smem_desc_sw128(s_p, 16, 1024);
+                const uint64_t vd = smem_desc_sw128(b0, kBox, 1024);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)   // 16 rows per MMA: +32 bytes of P lines, +2 KB of V lines
+                  mma_pair_f16_w(tmem + kColO + 128 * bb, pd + ((pg_i * kPChunk + ks * 32) >> 4),
+                                 vd + ((ks * 2048) >> 4), idO, (j | pg_i | ks) != 0);
+              }
               mma_commit_pair_w(empty, 0x3);
             }
           }
@@ -595,6 +639,39 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<F8>::kThr
         if (part == 0 && head < p.n_heads) p.lse_part[((size_t)r * p.n_heads + head) * S + s] = -INFINITY;
         continue;
       }
+      // D8: the scores are (q scale of the head) x (row scale) x the code
+      // GEMM; the weights of the value GEMM get each row's scale relative to
+      // the segment's largest (taken here from all of the segment's pages),
+      // times 16, and O is multiplied back in the epilogue
+      float slq = p.scale_log2, w_k = 0.f, o_back = 1.f;
+      if constexpr (D8) {
+        if (head < p.n_heads) slq *= __ldg(p.q_scale + (size_t)r * p.n_heads + head);
+        float smx = 0.f;
+        for (int i = 0; i < n_tiles; ++i) {
+          const int row0 = lo + kTile * i + 128 * half + 64 * ch;
+          const int nv = min(max(hi - row0, 0), 64);
+          if (nv > 0) {
+            bool pok;
+            const int pg = page_of(p, b, row0, &pok);
+            if (pok) {
+              if (lane < nv) smx = fmaxf(smx, __ldg(p.cache_scale + (size_t)pg * 64 + lane));
+              if (lane + 32 < nv) smx = fmaxf(smx, __ldg(p.cache_scale + (size_t)pg * 64 + 32 + lane));
+            }
+          }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) smx = fmaxf(smx, __shfl_xor_sync(0xffffffffu, smx, o));
+        // double-buffered by segment parity: a warp writes the next segment's
+        // slot only after this segment's later syncs, which follow every read here
+        float* scm = reinterpret_cast<float*>(misc + kMScMax) + (uc & 1) * kSoftWarps;
+        if (lane == 0) scm[warp - kWarpSoft0] = smx;
+        if (!(ok = soft_sync(1))) break;
+        float m8 = scm[0];
+#pragma unroll
+        for (int w = 1; w < kSoftWarps; ++w) m8 = fmaxf(m8, scm[w]);
+        w_k = m8 > 0.f ? kPScale8 / m8 : 0.f;
+        o_back = m8 / kPScale8;
+      }
       float m_run = -INFINITY, l_acc = 0.f;
       for (int i = 0; i < n_tiles; ++i) {
         const uint32_t t = gt + i;
@@ -610,7 +687,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<F8>::kThr
           if (!pok) {
             nvalid = 0;
             flag_error(p.err, MLA_DEVERR_PAGE);
-          } else if constexpr (F8) {
+          } else if constexpr (F8 || D8) {
             sc_lo = __ldg(p.cache_scale + (size_t)pg * 64 + lane);
             sc_hi = __ldg(p.cache_scale + (size_t)pg * 64 + 32 + lane);
           }
@@ -626,8 +703,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<F8>::kThr
         float mx = -INFINITY;
 #pragma unroll
         for (int j = 0; j < 64; ++j) {
-          float sl = p.scale_log2;
-          if constexpr (F8) sl *= __shfl_sync(0xffffffffu, j < 32 ? sc_lo : sc_hi, j & 31);
+          float sl = slq;
+          if constexpr (F8 || D8) sl *= __shfl_sync(0xffffffffu, j < 32 ? sc_lo : sc_hi, j & 31);
           v[j] = j < nvalid ? v[j] * sl : -INFINITY;
           mx = fmaxf(mx, v[j]);
         }
@@ -638,19 +715,39 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<F8>::kThr
         rm[part * kHPC + hh] = mx;
         if (!(ok = soft_sync(0))) break;
         const float tmax = fmaxf(fmaxf(rm[hh], rm[kHPC + hh]), fmaxf(rm[2 * kHPC + hh], rm[3 * kHPC + hh]));
-        const float m_new = (tmax > m_run + kRescaleLog2) ? tmax : m_run;
+        const float m_new = (tmax > m_run + (D8 ? kRescaleLog2Q8 : kRescaleLog2)) ? tmax : m_run;
         const bool changed = m_new != m_run;
         // factor for the sums and the accumulator kept so far (0 when nothing was kept)
         const float alpha = (m_run == -INFINITY) ? 0.f : exp2_approx(m_run - m_new);
         m_run = m_new;
         const float msub = m_new == -INFINITY ? 0.f : m_new;
-        uint32_t pk[32];
+        uint32_t pk[32];   // D8: pk[0..15] the hi codes of the 64 rows, pk[16..31] the lo codes
         float sum = 0.f;
+        if constexpr (D8) {
+          const float wlo = sc_lo * w_k, whi = sc_hi * w_k;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float p0 = exp2_approx(v[2 * j] - msub), p1 = exp2_approx(v[2 * j + 1] - msub);
-          sum += p0 + p1;
-          pk[j] = F8 ? pack_f16(p0, p1) : pack_bf16(p0, p1);
+          for (int j = 0; j < 32; ++j) {
+            const float p0 = exp2_approx(v[2 * j] - msub), p1 = exp2_approx(v[2 * j + 1] - msub);
+            sum += p0 + p1;
+            const float x0 = p0 * __shfl_sync(0xffffffffu, 2 * j < 32 ? wlo : whi, (2 * j) & 31);
+            const float x1 = p1 * __shfl_sync(0xffffffffu, 2 * j + 1 < 32 ? wlo : whi, (2 * j + 1) & 31);
+            uint32_t h2, l2;
+            split_e4m3x2(x0, x1, h2, l2);
+            if (j & 1) {
+              pk[j >> 1] |= h2 << 16;
+              pk[16 + (j >> 1)] |= l2 << 16;
+            } else {
+              pk[j >> 1] = h2;
+              pk[16 + (j >> 1)] = l2;
+            }
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float p0 = exp2_approx(v[2 * j] - msub), p1 = exp2_approx(v[2 * j + 1] - msub);
+            sum += p0 + p1;
+            pk[j] = F8 ? pack_f16(p0, p1) : pack_bf16(p0, p1);
+          }
         }
         l_acc = changed ? fmaf(l_acc, alpha, sum) : l_acc + sum;
         // every phase of o_done is observed in order (a parity wait cannot
@@ -675,8 +772,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<F8>::kThr
           }
         }
         // P of this thread's 64 rows (one page of the tile): line hh of the
-        // page's K-major [64 heads x 64 rows] tile, 128-byte swizzled
-        {
+        // page's K-major [64 heads x 64 rows] tile, 128-byte swizzled (D8: a
+        // 64-byte line in each of the hi and lo tiles, 64-byte swizzled)
+        if constexpr (D8) {
+#pragma unroll
+          for (int hl = 0; hl < 2; ++hl) {
+            uint8_t* line = s_pbuf + part * kPChunk + hl * kBox8 + hh * 64;
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              *reinterpret_cast<uint4*>(line + ((q ^ ((hh >> 1) & 3)) << 4)) =
+                  make_uint4(pk[16 * hl + 4 * q], pk[16 * hl + 4 * q + 1], pk[16 * hl + 4 * q + 2],
+                             pk[16 * hl + 4 * q + 3]);
+          }
+        } else {
           uint8_t* line = s_pbuf + part * kPChunk + hh * 128;
 #pragma unroll
           for (int q = 0; q < 8; ++q)
@@ -698,7 +806,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<F8>::kThr
       }
       if (ok) {
         const float lt = red_sum[hh] + red_sum[kHPC + hh] + red_sum[2 * kHPC + hh] + red_sum[3 * kHPC + hh];
-        const float inv_l = lt > 0.f ? 1.0f / lt : 0.f;
+        const float inv_l = lt > 0.f ? o_back / lt : 0.f;
         if (part == 0 && head < p.n_heads)
           p.lse_part[((size_t)r * p.n_heads + head) * S + s] =
               lt > 0.f ? (m_run + log2f(lt)) * 0.69314718055994531f : -INFINITY;
@@ -939,16 +1047,33 @@ bool claim_slot(const void* workspace, unsigned** claim, unsigned** done) {
 }  // namespace
 
 bool decode_pair_supported(const DecodeArgs& a) {
-  return a.q_dtype == MLA_BF16 && (a.cache_dtype == MLA_BF16 || a.cache_dtype == MLA_E4M3) && a.page_size == 64 &&
-         a.n_heads > 64 && a.n_heads <= 128 && (long long)a.batch * a.q_len * a.num_splits * 2 < (1ll << 31);
+  const bool forms = (a.q_dtype == MLA_BF16 && (a.cache_dtype == MLA_BF16 || a.cache_dtype == MLA_E4M3)) ||
+                     (a.q_dtype == MLA_E4M3 && a.cache_dtype == MLA_E4M3 && a.q_scale);
+  return forms && a.page_size == 64 && a.n_heads > 64 && a.n_heads <= 128 &&
+         (long long)a.batch * a.q_len * a.num_splits * 2 < (1ll << 31);
 }
 
 cudaError_t launch_decode_pair(const DecodeArgs& a, cudaStream_t st) {
   TensorMapEncodeFn enc = tensor_map_encoder();
   if (!enc) return cudaErrorNotSupported;
-  const bool f8 = a.cache_dtype == MLA_E4M3;
+  const bool d8 = a.q_dtype == MLA_E4M3;                  // two-term e4m3 query: 8-bit MMAs
+  const bool f8 = a.cache_dtype == MLA_E4M3 && !d8;       // bf16 query over e4m3: widened operands
   CUtensorMap tc, tc2, tq;
-  if (f8) {
+  if (d8) {
+    // the e4m3 pool as 2-D [num_pages * 9 * 64 lines x 64 codes] of 64-byte
+    // lines, 64-byte swizzled (the operand layout): boxes of one block and of
+    // two adjacent blocks
+    for (int k = 0; k < 2; ++k) {
+      cuuint64_t dims[2] = {64, (cuuint64_t)a.num_pages * kChunks * 64};
+      cuuint64_t strides[1] = {64};
+      cuuint32_t box[2] = {64, k == 0 ? 64u : 128u};
+      cuuint32_t es[2] = {1, 1};
+      if (enc(k == 0 ? &tc : &tc2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(a.cache), dims, strides, box,
+              es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    }
+  } else if (f8) {
     // the e4m3 pool as 2-D [num_pages * 9 * 64 lines x 64 codes] of 64-byte
     // lines, unswizzled (the converters swizzle): boxes of one block
     cuuint64_t dims[2] = {64, (cuuint64_t)a.num_pages * kChunks * 64};
@@ -974,7 +1099,19 @@ cudaError_t launch_decode_pair(const DecodeArgs& a, cudaStream_t st) {
         return cudaErrorInvalidValue;
     }
   }
-  {
+  if (d8) {
+    // the two-term query [rows, 2, heads, 576] codes as 3-D [2 rows planes x
+    // heads x 576]: boxes of 64 codes x 64 heads of one plane, 64-byte swizzled
+    // (heads past n_heads read as zeros)
+    cuuint64_t dims[3] = {MLA_D_ROW, (cuuint64_t)a.n_heads, (cuuint64_t)a.batch * a.q_len * 2};
+    cuuint64_t strides[2] = {MLA_D_ROW, (cuuint64_t)a.n_heads * MLA_D_ROW};
+    cuuint32_t box[3] = {64, (cuuint32_t)kHPC, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    if (enc(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(a.q_abs), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  } else {
     // q_abs [rows, heads, 576]: boxes of 64 columns x 64 heads of one row
     // (heads past n_heads read as zeros)
     cuuint64_t dims[3] = {MLA_D_ROW, (cuuint64_t)a.n_heads, (cuuint64_t)a.batch * a.q_len};
@@ -986,9 +1123,11 @@ cudaError_t launch_decode_pair(const DecodeArgs& a, cudaStream_t st) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  const int smem = f8 ? PairLayout<true>::kSmem : PairLayout<false>::kSmem;
-  cudaError_t e = f8 ? cudaFuncSetAttribute(decode_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)
-                     : cudaFuncSetAttribute(decode_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  const int smem = d8 ? PairLayout<false, true>::kSmem : f8 ? PairLayout<true>::kSmem : PairLayout<false>::kSmem;
+  cudaError_t e =
+      d8   ? cudaFuncSetAttribute(decode_pair_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)
+      : f8 ? cudaFuncSetAttribute(decode_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)
+           : cudaFuncSetAttribute(decode_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   // Runs of splits per claimed unit.  With at least four splits per CTA pair,
   // every pair gets one run of ceil(splits / pairs) consecutive splits: each
@@ -1003,9 +1142,12 @@ cudaError_t launch_decode_pair(const DecodeArgs& a, cudaStream_t st) {
   const long long units = (n_flat + run - 1) / run;
   PairParams p{a.n_heads, a.q_len, a.batch, a.block_table, a.max_pages, a.num_pages, a.seq_lens, a.num_splits,
                a.split_tokens, run, a.softmax_scale * 1.4426950408889634f, nullptr, nullptr, a.o_part, a.lse_part,
-               a.err, g_wait_limit.load(), g_withhold_q.load(), a.cache_scale};
+               a.err, g_wait_limit.load(), g_withhold_q.load(), a.cache_scale, a.q_scale};
   if (!claim_slot(a.o_part, &p.claim, &p.done)) return cudaErrorInvalidSymbol;
   const long long pairs = units < P ? units : P;
+  if (d8)
+    return launch_dependent(decode_pair_kernel<false, true>, dim3((unsigned)(2 * pairs)),
+                            dim3(PairLayout<false, true>::kThreads), smem, st, tc, tc2, tq, p);
   if (f8)
     return launch_dependent(decode_pair_kernel<true>, dim3((unsigned)(2 * pairs)), dim3(PairLayout<true>::kThreads),
                             smem, st, tc, tc2, tq, p);

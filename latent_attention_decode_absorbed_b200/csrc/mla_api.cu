@@ -171,6 +171,49 @@ mla_status mla_decode_fwd(const void* q_abs, mla_dtype q_dtype, const void* cach
   return cuda_status(launch_decode_simt(a, stream), "mla_decode_fwd launch");
 }
 
+mla_status mla_split_q_e4m3(const void* q_abs, int rows, int n_heads, void* q8, float* q_scale,
+                            cudaStream_t stream) {
+  MLA_REQUIRE(rows >= 0, MLA_ERR_INVALID_ARG, "mla_split_q_e4m3: rows < 0");
+  MLA_REQUIRE(n_heads >= 1 && n_heads <= MLA_MAX_HEADS, MLA_ERR_INVALID_ARG,
+              "mla_split_q_e4m3: n_heads must be in [1, %d]", MLA_MAX_HEADS);
+  MLA_REQUIRE((long long)rows * n_heads * 32 < (1ll << 31), MLA_ERR_UNSUPPORTED, "mla_split_q_e4m3: too many rows");
+  if (rows == 0) return MLA_OK;
+  MLA_REQUIRE(q_abs && q8 && q_scale, MLA_ERR_INVALID_ARG, "mla_split_q_e4m3: null pointer");
+  MLA_REQUIRE(aligned(q_abs, 16) && aligned(q8, 16) && aligned(q_scale, 4), MLA_ERR_INVALID_ARG,
+              "mla_split_q_e4m3: q_abs and q8 must be 16-byte aligned");
+  return cuda_status(launch_split_q_e4m3(q_abs, rows, n_heads, q8, q_scale, stream), "mla_split_q_e4m3 launch");
+}
+
+mla_status mla_decode_fwd_q8(const void* q8, const float* q_scale, const void* cache, const float* cache_scale,
+                             int num_pages, const int32_t* block_table, int max_pages_per_seq, int page_size,
+                             const int32_t* seq_lens, int batch, int q_len, int n_heads, int num_splits,
+                             int split_tokens, float softmax_scale, float* o_part, float* lse_part,
+                             int32_t* err_word, cudaStream_t stream) {
+  MLA_REQUIRE(page_size == MLA_PAGE, MLA_ERR_UNSUPPORTED, "mla_decode_fwd_q8: page_size must be %d", MLA_PAGE);
+  MLA_REQUIRE(batch >= 1 && q_len >= 1 && num_pages >= 1 && max_pages_per_seq >= 1, MLA_ERR_INVALID_ARG,
+              "mla_decode_fwd_q8: batch, q_len, num_pages, max_pages_per_seq must be >= 1");
+  MLA_REQUIRE(n_heads > 64 && n_heads <= MLA_MAX_HEADS, MLA_ERR_UNSUPPORTED,
+              "mla_decode_fwd_q8: n_heads must be in [65, %d]", MLA_MAX_HEADS);
+  MLA_REQUIRE(num_splits >= 1 && split_tokens >= page_size && split_tokens % page_size == 0,
+              MLA_ERR_INVALID_ARG, "mla_decode_fwd_q8: need num_splits >= 1 and split_tokens a positive multiple of page_size");
+  MLA_REQUIRE((long long)num_splits * split_tokens >= (long long)max_pages_per_seq * page_size,
+              MLA_ERR_INVALID_ARG, "mla_decode_fwd_q8: num_splits * split_tokens must cover max_pages_per_seq * page_size");
+  MLA_REQUIRE((long long)max_pages_per_seq * page_size < (1ll << 31), MLA_ERR_INVALID_ARG,
+              "mla_decode_fwd_q8: table capacity overflows int32 positions");
+  MLA_REQUIRE(isfinite(softmax_scale) && softmax_scale > 0.f, MLA_ERR_INVALID_ARG,
+              "mla_decode_fwd_q8: softmax_scale must be finite and > 0");
+  MLA_REQUIRE(q8 && q_scale && cache && cache_scale && block_table && seq_lens && o_part && lse_part,
+              MLA_ERR_INVALID_ARG, "mla_decode_fwd_q8: null pointer");
+  MLA_REQUIRE(aligned(q8, 16) && aligned(cache, 128) && aligned(o_part, 16), MLA_ERR_INVALID_ARG,
+              "mla_decode_fwd_q8: q8 and o_part must be 16-byte aligned, cache 128-byte aligned");
+  MLA_REQUIRE((long long)batch * q_len <= 65535, MLA_ERR_UNSUPPORTED, "mla_decode_fwd_q8: batch*q_len above 65535");
+  DecodeArgs a{q8, MLA_E4M3, cache, cache_scale, MLA_E4M3, num_pages, block_table, max_pages_per_seq,
+               page_size, seq_lens, batch, q_len, n_heads, num_splits, split_tokens, softmax_scale,
+               o_part, lse_part, err_word, q_scale};
+  MLA_REQUIRE(decode_pair_supported(a), MLA_ERR_UNSUPPORTED, "mla_decode_fwd_q8: unsupported sizes");
+  return cuda_status(launch_decode_pair(a, stream), "mla_decode_fwd_q8 launch (tcgen05 kind::f8f6f4, head-split pairs)");
+}
+
 mla_status mla_out_proj(const void* out, const void* w_o, float* u, int rows, int n_heads, int d_model,
                         cudaStream_t stream) {
   MLA_REQUIRE(rows >= 0, MLA_ERR_INVALID_ARG, "mla_out_proj: rows < 0");

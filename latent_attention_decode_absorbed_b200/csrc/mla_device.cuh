@@ -88,4 +88,16 @@ __device__ __forceinline__ void load16(const __nv_bfloat16* p, float* v) {
   }
 }
 
+// Two-term e4m3 form of (x0, x1): hi = e4m3(x), lo = e4m3(x - hi) (the
+// difference is exact in fp32), both round-to-nearest-even and saturating;
+// each pair packed with x0's code in the low byte.
+__device__ __forceinline__ void split_e4m3x2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  const __nv_fp8x2_storage_t h = __nv_cvt_float2_to_fp8x2(make_float2(x0, x1), __NV_SATFINITE, __NV_E4M3);
+  const float2 b = __half22float2(__half2(__nv_cvt_fp8x2_to_halfraw2(h, __NV_E4M3)));
+  const __nv_fp8x2_storage_t l =
+      __nv_cvt_float2_to_fp8x2(make_float2(x0 - b.x, x1 - b.y), __NV_SATFINITE, __NV_E4M3);
+  hi = h;
+  lo = l;
+}
+
 }  // namespace mla

@@ -27,6 +27,8 @@ struct AppendArgs {
 };
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t st);
 
+// the two-term e4m3 form of bf16 absorbed queries (see mla_split_q_e4m3)
+cudaError_t launch_split_q_e4m3(const void* q_abs, int rows, int n_heads, void* q8, float* q_scale, cudaStream_t st);
 cudaError_t launch_absorb_q(const void* q_nope, const void* q_pe, const void* w_uk, void* q_abs,
                             int rows, int n_heads, int dtype, cudaStream_t st);
 cudaError_t launch_out_uv(const void* o_lat, const void* w_uv, void* out, int rows, int n_heads,
@@ -43,9 +45,11 @@ struct DecodeArgs {
   const int32_t* seq_lens; int batch; int q_len; int n_heads;
   int num_splits; int split_tokens; float softmax_scale;
   float* o_part; float* lse_part; int32_t* err;
+  const float* q_scale;   // q_dtype E4M3: the two-term query's scale per (row, head)
 };
 cudaError_t launch_decode_simt(const DecodeArgs& a, cudaStream_t st);
-// tcgen05 path for 65..128 heads over a bf16 cache (heads split across a CTA pair)
+// tcgen05 path for 65..128 heads (heads split across a CTA pair): bf16 queries over
+// a bf16 or e4m3 cache, or the two-term e4m3 query over an e4m3 cache (8-bit MMAs)
 bool decode_pair_supported(const DecodeArgs& a);
 cudaError_t launch_decode_pair(const DecodeArgs& a, cudaStream_t st);
 // tcgen05 path: bf16 queries over a bf16 or e4m3 cache

@@ -249,6 +249,18 @@ __device__ __forceinline__ void mma_pair_f16_w(uint32_t d_tmem, uint64_t a_desc,
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// The same for e4m3 A and B (kind::f8f6f4): one K=32 step (32 bytes along
+// a K-major line, 32 rows of an MN-major tile).
+__device__ __forceinline__ void mma_pair_e4m3_w(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 // D[tmem] (+)= A[tmem] * B[smem]^T over one K=16 step for the pair, issued
 // by a converged warp (A from tensor memory: for M = 128 each CTA's 64 A rows
 // sit in lanes 0-63 of its own TMEM, 16 bf16 of K in 8 columns).
@@ -365,11 +377,35 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr, uint32_t lbo,
   return d;
 }
 
+// The same with a 64-byte swizzle (8-row x 64-byte atoms, 512-byte aligned),
+// for 8-bit tiles whose lines are 64 bytes:
+//   K-major : rows are 64-byte lines of 64 K-elements; `sbo` = 8-row group stride.
+//   MN-major: each line holds 64 consecutive M/N elements of one K index;
+//             `sbo` = 8-K-row group stride, `lbo` = 64-element M/N block stride.
+__device__ __forceinline__ uint64_t smem_desc_sw64(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((addr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+  d |= 1ull << 46;   // descriptor version for sm_100
+  d |= 4ull << 61;   // 64-byte swizzle
+  return d;
+}
+
 // Instruction descriptor for kind::f16 with bf16 (or f16) A/B and fp32 D.
 __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool a_mn_major, bool b_mn_major, bool f16 = false) {
   return (1u << 4)                                   // D format: f32
          | ((f16 ? 0u : 1u) << 7)                    // A format: bf16 (1) / f16 (0)
          | ((f16 ? 0u : 1u) << 10)                   // B format
+         | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
+         (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// Instruction descriptor for kind::f8f6f4 with e4m3 A and B (format code 0)
+// and fp32 D; MN-major is allowed for e4m3 operands.
+__host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N, bool a_mn_major, bool b_mn_major) {
+  return (1u << 4)                                   // D format: f32
+         | (0u << 7) | (0u << 10)                    // A, B format: e4m3
          | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
          (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }

@@ -16,7 +16,7 @@ import math
 import numpy as np
 
 from . import (D_C, D_R, D_ROW, D_V, MLA_BF16, MLA_E4M3, MLA_F32, PAGE, mla_absorb_q, mla_cache_append,
-               mla_combine, mla_combine_out_uv, mla_decode_fwd, mla_kv_proj_append, mla_kv_proj_workspace_bytes, mla_out_proj,
+               mla_combine, mla_combine_out_uv, mla_decode_fwd, mla_decode_fwd_q8, mla_split_q_e4m3, mla_kv_proj_append, mla_kv_proj_workspace_bytes, mla_out_proj,
                mla_out_uv, mla_rope_table)
 
 _DT = {"f32": MLA_F32, "bf16": MLA_BF16, "e4m3": MLA_E4M3}
@@ -35,7 +35,7 @@ class DecodeStep:
 
     def __init__(self, *, batch, q_len, n_heads, dtype, cache_dtype, block_table, num_pages,
                  split_tokens, max_pos=None, theta=10000.0, eps=1e-6, norm_gain=None,
-                 softmax_scale=None, device="cuda"):
+                 softmax_scale=None, device="cuda", q8=None):
         import torch
         self.torch = torch
         self.batch, self.q_len, self.n_heads = int(batch), int(q_len), int(n_heads)
@@ -66,6 +66,15 @@ class DecodeStep:
         rows = self.batch * self.q_len
         qdt = _torch_dtype(self.dtype)
         self.q_abs = torch.empty((rows, self.n_heads, D_ROW), dtype=qdt, device=dev)
+        # e4m3 cache, bf16 queries, 65..128 heads: both GEMMs on 8-bit MMAs from
+        # the query's two-term e4m3 form (q8=False keeps the widened f16 operands)
+        q8_ok = self.cache_dtype == MLA_E4M3 and self.dtype == MLA_BF16 and 64 < self.n_heads <= 128
+        if q8 and not q8_ok:
+            raise ValueError("q8 needs an e4m3 cache, bf16 queries and 65..128 heads")
+        self.q8 = q8_ok if q8 is None else bool(q8)
+        self.q_e4m3 = (torch.empty((rows, 2, self.n_heads, D_ROW), dtype=torch.uint8, device=dev)
+                       if self.q8 else None)
+        self.q_scale = torch.empty((rows, self.n_heads), dtype=torch.float32, device=dev) if self.q8 else None
         self.o_part = torch.empty((rows, self.n_heads, self.num_splits, D_C), dtype=torch.float32, device=dev)
         self.lse_part = torch.empty((rows, self.n_heads, self.num_splits), dtype=torch.float32, device=dev)
         self.o_lat = torch.empty((rows, self.n_heads, D_C), dtype=qdt, device=dev)
@@ -82,9 +91,18 @@ class DecodeStep:
                          self.cache, self.cache_scale, self.cache_dtype, self.num_pages, self.err, stream)
 
     def absorb(self, q_nope, q_pe, w_uk, stream=None):
+        """q_abs = [W_UK^T q_nope; q_pe]; with q8 also its two-term e4m3 form."""
         mla_absorb_q(q_nope, q_pe, w_uk, self.q_abs, self.batch * self.q_len, self.n_heads, self.dtype, stream)
+        if self.q8:
+            mla_split_q_e4m3(self.q_abs, self.batch * self.q_len, self.n_heads, self.q_e4m3, self.q_scale, stream)
 
     def attend(self, stream=None):
+        if self.q8:
+            mla_decode_fwd_q8(self.q_e4m3, self.q_scale, self.cache, self.cache_scale, self.num_pages,
+                              self.block_table, self.max_pages, PAGE, self.seq_lens, self.batch, self.q_len,
+                              self.n_heads, self.num_splits, self.split_tokens, self.softmax_scale, self.o_part,
+                              self.lse_part, self.err, stream)
+            return
         mla_decode_fwd(self.q_abs, self.dtype, self.cache, self.cache_scale, self.cache_dtype, self.num_pages,
                        self.block_table, self.max_pages, PAGE, self.seq_lens, self.batch, self.q_len,
                        self.n_heads, self.num_splits, self.split_tokens, self.softmax_scale, self.o_part,
@@ -119,7 +137,7 @@ class DecodeStep:
 
     @property
     def launches_per_step(self):
-        return 4 if self.fused_post else 5
+        return (4 if self.fused_post else 5) + (1 if self.q8 else 0)
 
     # -- the projections on either side of the path ---------------------------
     def append_from_hidden(self, h, w_kva, seq_ids, positions, stream=None):

@@ -152,6 +152,28 @@ def dequantize_rows_e4m3(codes: np.ndarray, scale: np.ndarray) -> np.ndarray:
     return e4m3_decode(codes) * np.asarray(scale, dtype=np.float64)[:, None]
 
 
+def split_query_e4m3(q: np.ndarray) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """Two-term e4m3 form of absorbed queries q [..., 576] (fp32 values):
+    the query operand of the 8-bit tensor-core decode over an e4m3 cache.
+
+    Not a step of the pages: with an e4m3 cache ([DENIZ] cache section,
+    [OCP-FP8]) both operands of an 8-bit MMA are 8-bit, so the query is
+    carried as two e4m3 terms on one fp32 scale per (row, head), in fp32:
+        a = max |q|;  inv = fp32(448 / a) (0 when a = 0);  y = fp32(q * inv)
+        hi = e4m3(y);  lo = e4m3(y - hi)   (y - hi is exact in fp32)
+        scale = fp32(a / 448)
+    so that q ~ scale * (hi + lo) to about 2^-8 relative.
+    Returns (hi codes, lo codes) uint8 [..., 576] and scale float32 [...]."""
+    q32 = np.asarray(q, dtype=np.float32)
+    a = np.max(np.abs(q32), axis=-1)
+    inv = np.where(a > 0, np.float32(E4M3_MAX) / np.where(a > 0, a, np.float32(1)), np.float32(0)).astype(np.float32)
+    y = (q32 * inv[..., None]).astype(np.float32)
+    hi = e4m3_encode(y.astype(np.float64))
+    lo = e4m3_encode(y.astype(np.float64) - e4m3_decode(hi))
+    scale = (a / np.float32(E4M3_MAX)).astype(np.float32)
+    return hi, lo, scale
+
+
 # --------------------------------------------------------------------------
 # cache write: RMSNorm on the latent, RoPE on the shared rope key
 # --------------------------------------------------------------------------

@@ -160,6 +160,40 @@ def pin_e4m3():
     assert np.all(z == 0) and zs[0] == 0.0
 
 
+def pin_split_query_e4m3():
+    """hi is a nearest e4m3 value to y = fp32(q * fp32(448 / max|q|)) and lo a
+    nearest to y - hi, checked by exhaustive search over every finite code
+    (tie-breaking is pinned by pin_e4m3); the absmax element maps to +-448;
+    hi + lo carries y to max(2^-8 |y|, 2^-10)."""
+    g = _rng(41)
+    vals = oracle.e4m3_decode(np.arange(256, dtype=np.uint8))
+    table = vals[~np.isnan(vals)]
+
+    def nearest_dist(x):
+        return np.min(np.abs(x[:, None] - table[None, :]), axis=1)
+
+    q = (g.standard_normal((3, 5, 576)) * np.exp(g.uniform(-4, 4, (3, 5, 1)))).astype(np.float32)
+    q[0, 1, :] = 0.0                                   # a zero (row, head)
+    hi, lo, sc = oracle.split_query_e4m3(q)
+    assert hi.shape == q.shape and lo.shape == q.shape and sc.shape == (3, 5)
+    a = np.abs(q).max(-1)
+    inv = np.where(a > 0, np.float32(448.0) / np.where(a > 0, a, np.float32(1)), np.float32(0)).astype(np.float32)
+    yf = (q * inv[..., None]).astype(np.float32).astype(np.float64).reshape(-1)
+    vh, vl = oracle.e4m3_decode(hi).reshape(-1), oracle.e4m3_decode(lo).reshape(-1)
+    assert np.all(np.abs(yf - vh) <= nearest_dist(yf) + 1e-12)
+    r = yf - vh
+    assert np.all(np.abs(r - vl) <= nearest_dist(r) + 1e-15)
+    err = np.abs(yf - vh - vl)
+    assert np.all(err <= np.maximum(2.0 ** -8 * np.abs(yf), 2.0 ** -10))
+    am = np.argmax(np.abs(q), axis=-1)
+    top = np.take_along_axis(np.abs(oracle.e4m3_decode(hi)), am[..., None], -1)[..., 0]
+    assert np.all(top[a > 0] == 448.0)
+    np.testing.assert_allclose(sc, a / 448.0, rtol=2.0 ** -23)
+    assert np.all(hi[0, 1] == 0) and np.all(lo[0, 1] == 0) and sc[0, 1] == 0.0
+    # q ~ scale * (hi + lo) to about 2^-8 of max|q| per element
+    rec = sc[..., None].astype(np.float64) * (oracle.e4m3_decode(hi) + oracle.e4m3_decode(lo))
+    assert np.max(np.abs(rec - q) / np.maximum(a[..., None], 1e-30)) <= 2.0 ** -8 * 1.01
+
 def pin_bf16_rounding():
     import torch
     g = _rng(4)
@@ -430,4 +464,5 @@ def pin_decompress_kv():
 ALL_PINS = [pin_cache_arithmetic, pin_rmsnorm, pin_rope, pin_e4m3, pin_bf16_rounding,
             pin_naive_equals_absorbed, pin_single_row, pin_uniform_scores, pin_two_rows_sigmoid,
             pin_row_permutation, pin_causal, pin_brute_force, pin_split_combine, pin_cache_rows,
-            pin_normwise_rel_err, pin_out_projection, pin_kv_a_projection, pin_decompress_kv]
+            pin_normwise_rel_err, pin_out_projection, pin_kv_a_projection, pin_decompress_kv,
+            pin_split_query_e4m3]

@@ -13,7 +13,8 @@ import pins
 ORIG = {name: getattr(om, name) for name in
         ["attention_naive", "attention_absorbed", "rope_angles", "rope", "rms_norm",
          "e4m3_encode", "combine_partials", "absorb_q", "out_uv", "round_to_bf16",
-          "normwise_rel_err", "out_projection", "kv_a_projection", "decompress_kv"]}
+          "normwise_rel_err", "out_projection", "kv_a_projection", "decompress_kv",
+          "split_query_e4m3"]}
 
 
 def _patch(monkeypatch, name, fn):
@@ -153,11 +154,26 @@ def _decompress_heads_reversed(monkeypatch):
     _patch(monkeypatch, "decompress_kv", dec)
 
 
+
+def _split_lo_own_scale(monkeypatch):
+    def split(q):
+        hi, lo, sc = ORIG["split_query_e4m3"](q)
+        y = om.e4m3_decode(lo) * 16.0                              # lo kept on a scale 16x finer
+        return hi, om.e4m3_encode(y), sc
+    _patch(monkeypatch, "split_query_e4m3", split)
+
+
+def _split_scale_inverted(monkeypatch):
+    def split(q):
+        hi, lo, sc = ORIG["split_query_e4m3"](q)
+        return hi, lo, np.where(sc > 0, 1.0 / np.where(sc > 0, sc, 1.0), 0.0).astype(np.float32)
+    _patch(monkeypatch, "split_query_e4m3", split)
+
 MUTATIONS = [_drop_rope_term, _scale_128, _rope_wrong_direction, _rope_half_split, _rms_no_sqrt,
              _causal_excludes_self, _e4m3_ties_away, _combine_no_weights, _wrong_value_matrix,
              _bf16_truncates, _gate_mean, _gate_den_from_got, _gate_wrong_axis, _gate_zero,
              _gate_global_norm, _concat_interleaved, _kv_a_transposed_halves, _decompress_swapped,
-             _decompress_heads_reversed]
+             _decompress_heads_reversed, _split_lo_own_scale, _split_scale_inverted]
 
 
 @pytest.mark.parametrize("mutate", MUTATIONS, ids=lambda f: f.__name__.strip("_"))
