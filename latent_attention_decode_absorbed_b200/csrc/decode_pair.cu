@@ -82,7 +82,8 @@ constexpr int kWarpConv0 = kWarpSoft0 + kSoftWarps, kConvWarps = 4;   // e4m3 ca
 constexpr int kQN = 8;                    // unit queue depth
 constexpr float kRescaleLog2 = 8.0f;      // lazy rescale threshold (log2 units)
 constexpr float kRescaleLog2Q8 = 4.0f;    // 8-bit MMAs: probabilities stay <= 2^4, and times
-constexpr float kPScale8 = 16.0f;         // 16 x (row scale / segment's largest) <= 256 < 448
+constexpr float kPScale8 = 16.0f;         // 16 x row scale / reference <= 16 x 1.75 ...
+constexpr float kScaleSlack8 = 1.75f;     // ... the reference is raised past 1.75x: <= 448
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;             // S of tile t at kColS + 128 (t & 1)
 constexpr uint32_t kColO = 256;           // O: dims 0..255 at 256, dims 256..511 at 384
@@ -95,8 +96,8 @@ constexpr int kMRedMax = kMTmem + 16;     // float [2 tile parities][2 lane halv
 constexpr int kMRedSum = kMRedMax + 2 * 4 * kHPC * 4;   // float [2 lane halves][2 column halves][64 heads]
 constexpr int kMUnitQ = kMRedSum + 4 * kHPC * 4;
 constexpr int kMStgSeq = kMUnitQ + 4 * kQN;   // int [8]: e4m3, the stage each staging slot was last filled for
-constexpr int kMScMax = kMStgSeq + 4 * 8;     // float [2 segment parities][8 softmax warps]: 8-bit MMAs
-constexpr int kMiscBytes = kMScMax + 4 * 2 * kSoftWarps;
+constexpr int kMRedSc = kMStgSeq + 4 * 8;    // float [2 tile parities][8 softmax warps]: 8-bit MMAs
+constexpr int kMiscBytes = kMRedSc + 4 * 2 * kSoftWarps;
 
 // Shared memory, barriers and threads of the bf16 (F8 = D8 = false), the
 // widening e4m3 (F8) and the 8-bit MMA e4m3 (D8) kernels.  With F8 the
@@ -217,6 +218,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<F8, D8>::
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + kMAbort);
   float* red_max = reinterpret_cast<float*>(misc + kMRedMax);
   float* red_sum = reinterpret_cast<float*>(misc + kMRedSum);
+  float* red_sc = reinterpret_cast<float*>(misc + kMRedSc);
   int* unit_q = reinterpret_cast<int*>(misc + kMUnitQ);
   uint8_t* s_pbuf = smem + kOffP;
   const uint32_t s_p = s_base + kOffP;
@@ -640,37 +642,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<F8, D8>::
         continue;
       }
       // D8: the scores are (q scale of the head) x (row scale) x the code
-      // GEMM; the weights of the value GEMM get each row's scale relative to
-      // the segment's largest (taken here from all of the segment's pages),
-      // times 16, and O is multiplied back in the epilogue
-      float slq = p.scale_log2, w_k = 0.f, o_back = 1.f;
+      // GEMM.  The weights of the value GEMM carry each row's scale relative
+      // to a reference s_ref, times 16: s_ref is the largest row scale seen so
+      // far in the segment, raised (with O rescaled) only when a tile's rows
+      // exceed it by 1.75x, so every weight stays <= 16 x 16 x 1.75 = 448.
+      // O is multiplied by s_ref / 16 in the epilogue.
+      float slq = p.scale_log2, s_ref = 0.f;
       if constexpr (D8) {
         if (head < p.n_heads) slq *= __ldg(p.q_scale + (size_t)r * p.n_heads + head);
-        float smx = 0.f;
-        for (int i = 0; i < n_tiles; ++i) {
-          const int row0 = lo + kTile * i + 128 * half + 64 * ch;
-          const int nv = min(max(hi - row0, 0), 64);
-          if (nv > 0) {
-            bool pok;
-            const int pg = page_of(p, b, row0, &pok);
-            if (pok) {
-              if (lane < nv) smx = fmaxf(smx, __ldg(p.cache_scale + (size_t)pg * 64 + lane));
-              if (lane + 32 < nv) smx = fmaxf(smx, __ldg(p.cache_scale + (size_t)pg * 64 + 32 + lane));
-            }
-          }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) smx = fmaxf(smx, __shfl_xor_sync(0xffffffffu, smx, o));
-        // double-buffered by segment parity: a warp writes the next segment's
-        // slot only after this segment's later syncs, which follow every read here
-        float* scm = reinterpret_cast<float*>(misc + kMScMax) + (uc & 1) * kSoftWarps;
-        if (lane == 0) scm[warp - kWarpSoft0] = smx;
-        if (!(ok = soft_sync(1))) break;
-        float m8 = scm[0];
-#pragma unroll
-        for (int w = 1; w < kSoftWarps; ++w) m8 = fmaxf(m8, scm[w]);
-        w_k = m8 > 0.f ? kPScale8 / m8 : 0.f;
-        o_back = m8 / kPScale8;
       }
       float m_run = -INFINITY, l_acc = 0.f;
       for (int i = 0; i < n_tiles; ++i) {
@@ -713,6 +692,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<F8, D8>::
         // sync, so no warp can overwrite a slot that another is still reading
         float* rm = red_max + sb * 4 * kHPC;
         rm[part * kHPC + hh] = mx;
+        if constexpr (D8) {   // the largest scale of this warp's visible rows, same buffering
+          float tsm = fmaxf(lane < nvalid ? sc_lo : 0.f, lane + 32 < nvalid ? sc_hi : 0.f);
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) tsm = fmaxf(tsm, __shfl_xor_sync(0xffffffffu, tsm, o));
+          if (lane == 0) red_sc[sb * kSoftWarps + (warp - kWarpSoft0)] = tsm;
+        }
         if (!(ok = soft_sync(0))) break;
         const float tmax = fmaxf(fmaxf(rm[hh], rm[kHPC + hh]), fmaxf(rm[2 * kHPC + hh], rm[3 * kHPC + hh]));
         const float m_new = (tmax > m_run + (D8 ? kRescaleLog2Q8 : kRescaleLog2)) ? tmax : m_run;
@@ -721,6 +706,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<F8, D8>::
         const float alpha = (m_run == -INFINITY) ? 0.f : exp2_approx(m_run - m_new);
         m_run = m_new;
         const float msub = m_new == -INFINITY ? 0.f : m_new;
+        float w_k = 0.f, s_fac = 1.f;   // D8: weight factor 16 / s_ref; O's factor for a raised s_ref
+        bool s_up = false;
+        if constexpr (D8) {
+          const float* rs = red_sc + sb * kSoftWarps;
+          float tsmax = rs[0];
+#pragma unroll
+          for (int w = 1; w < kSoftWarps; ++w) tsmax = fmaxf(tsmax, rs[w]);
+          if (tsmax > kScaleSlack8 * s_ref) {
+            s_up = s_ref > 0.f;
+            s_fac = s_up ? s_ref / tsmax : 1.f;
+            s_ref = tsmax;
+          }
+          w_k = s_ref > 0.f ? kPScale8 / s_ref : 0.f;
+        }
         uint32_t pk[32];   // D8: pk[0..15] the hi codes of the 64 rows, pk[16..31] the lo codes
         float sum = 0.f;
         if constexpr (D8) {
@@ -757,8 +756,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<F8, D8>::
           ok = __all_sync(0xffffffffu, mbar_wait<false>(bar(kBODone), (t - 1) & 1, abort_flag, lim));
           if (!ok) break;
           tc_fence_after();
-          if (__any_sync(0xffffffffu, changed)) {
-            const float f = changed ? alpha : 1.f;
+          if (s_up || __any_sync(0xffffffffu, changed)) {
+            const float f = (changed ? alpha : 1.f) * s_fac;
             const uint32_t oc = tmem + lane_addr + kColO + 128 * ch;
 #pragma unroll 1
             for (int c4 = 0; c4 < 4; ++c4) {
@@ -806,7 +805,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<F8, D8>::
       }
       if (ok) {
         const float lt = red_sum[hh] + red_sum[kHPC + hh] + red_sum[2 * kHPC + hh] + red_sum[3 * kHPC + hh];
-        const float inv_l = lt > 0.f ? o_back / lt : 0.f;
+        const float inv_l = lt > 0.f ? (D8 ? s_ref / kPScale8 : 1.f) / lt : 0.f;
         if (part == 0 && head < p.n_heads)
           p.lse_part[((size_t)r * p.n_heads + head) * S + s] =
               lt > 0.f ? (m_run + log2f(lt)) * 0.69314718055994531f : -INFINITY;
