@@ -261,13 +261,14 @@ mla_status mla_split_q_e4m3(const void* q_abs, int rows, int n_heads, void* q8, 
  * conventions (o_part, lse_part, merged runs of splits, pool contract,
  * concurrency rule) with the query given in the two-term form of
  * mla_split_q_e4m3.  The scores are q_scale[r,h] * cache_scale[j] * the code
- * GEMM of (hi + lo) with row j's codes; the value GEMM's weights are carried
- * as two e4m3 terms too, with each row's scale folded in relative to the
- * largest scale among the rows of the unit of work, so that o_part holds
+ * GEMM of (hi + lo) with row j's codes.  The value GEMM's weights are carried
+ * as two e4m3 terms too: e^{z_j - m} * cache_scale[j] / s_ref * 16, where the
+ * running maximum m is raised once a tile's scores exceed it by 4 (log2
+ * units) and the reference s_ref is the largest row scale seen so far in the
+ * unit of work, raised once a tile's scales exceed it by 1.75x (O rescaled
+ * by the same factor), so every weight stays <= 448.  o_part then holds
  *   sum_j e^{z_j - m} (codes_j * cache_scale[j])[0:512] / sum_j e^{z_j - m}
- * to within about 2^-8 relative per weight.  The running maximum m is
- * raised once a tile's scores exceed it by 4 (log2 units), which keeps each
- * weight below 448.
+ * to within about 2^-8 relative per weight.
  *   q8, q_scale  from mla_split_q_e4m3 for batch*q_len rows and n_heads
  *   other arguments as for mla_decode_fwd with cache_dtype E4M3
  * Supported: page_size 64, 65 <= n_heads <= 128 (else MLA_ERR_UNSUPPORTED).

@@ -1,8 +1,15 @@
 // Split-KV latent attention for 65..128 heads over a bf16 or e4m3 cache, on
 // the tcgen05 tensor cores, with the heads split between the two CTAs of a
-// pair.  With an e4m3 cache (the F8 instantiation) converter warps widen the
-// staged codes into the same f16 operand layout, Q and P are f16, and the
-// softmax applies each row's dequantisation scale to its scores.
+// pair.  Three instantiations:
+//   bf16 cache, bf16 Q and P (kind::f16);
+//   F8: e4m3 cache with bf16 queries: converter warps widen the staged codes
+//       into the same f16 operand layout, Q and P are f16, and the softmax
+//       applies each row's dequantisation scale to its scores;
+//   D8: e4m3 cache with the query in two e4m3 terms (hi + lo on one scale
+//       per head): both GEMMs on kind::f8f6f4 straight from the cache codes,
+//       64-byte swizzled stages of half the size (twice as many), the
+//       softmax weights written as two e4m3 terms with each row's scale
+//       folded in relative to a running reference.
 //
 // What it computes ("DeepSeek-V2: MLA Explained", "MLA Full Formulas" part 3
 // with the absorption of "Optimization Note"): for each head h of query row
