@@ -313,7 +313,7 @@ def run_gpu(args, w, rank, world, local_rank):
     from workloads.device import DeviceWorkload
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    dw = DeviceWorkload(w, device=dev)
+    dw = DeviceWorkload(w, device=dev, q8=False if args.f16_operands else None)
     step = dw.step
     lens = dw.lens
     stream = torch.cuda.current_stream(dev)
@@ -471,7 +471,7 @@ def time_extra(args, name, dev, stream):
     import torch
     from workloads.device import DeviceWorkload
     w = W.WORKLOADS[name]
-    dw = DeviceWorkload(w, device=dev)
+    dw = DeviceWorkload(w, device=dev, q8=False if args.f16_operands else None)
     step = dw.step
     alg_bytes, alg_flops = algorithmic(w, dw.lens)
     flush = torch.empty(int(256e6) // 4, dtype=torch.float32, device=dev) if alg_bytes <= 256e6 else None
@@ -523,6 +523,8 @@ def main():
     ap.add_argument("--batch", type=int, default=None, help="override the workload's batch (profiling)")
     ap.add_argument("--seq-len", type=int, default=None, help="override the workload's fixed length (profiling)")
     ap.add_argument("--split-tokens", type=int, default=None, help="override the split length (profiling)")
+    ap.add_argument("--f16-operands", action="store_true",
+                    help="e4m3 cache: the widened f16-operand decode (mla_decode_fwd) instead of the 8-bit MMAs (profiling)")
     args = ap.parse_args()
     assert args.warmup >= 3, "at least 3 warm-up steps"
     rank = int(os.environ.get("RANK", 0))

@@ -28,7 +28,7 @@ def to_host_f64(t) -> np.ndarray:
 class DeviceWorkload:
     """A workload's weights, step inputs and a filled cache on the GPU."""
 
-    def __init__(self, w: Workload, split_tokens=None, device="cuda", build_cache=True, norm_gain=None):
+    def __init__(self, w: Workload, split_tokens=None, device="cuda", build_cache=True, norm_gain=None, q8=None):
         import torch
         from latent_attention_decode_absorbed_b200 import DecodeStep
         self.w = w
@@ -38,7 +38,7 @@ class DeviceWorkload:
                                cache_dtype=w.cache_dtype, block_table=self.bt, num_pages=self.num_pages,
                                split_tokens=split_tokens or w.split_tokens, max_pos=int(self.lens.max()),
                                theta=w.theta, eps=w.eps, norm_gain=norm_gain, softmax_scale=w.softmax_scale,
-                               device=device)
+                               device=device, q8=q8)
         self.step.seq_lens.copy_(torch.from_numpy(self.lens))
         qn, qp = queries(w)
         wuk, wuv = weights(w)
