@@ -154,3 +154,44 @@ def test_decode_workspace_bytes_host(lib):
     assert mla.mla_decode_workspace_bytes(128, 2, 128, 4) == 256 * 128 * 4 * 513 * 4
     assert mla.mla_decode_workspace_bytes(0, 1, 128, 4) == 0
     assert mla.mla_decode_workspace_bytes(1, 1, 16, -1) == 0
+
+
+def _q8_kwargs(**over):
+    kw = dict(q8=FAKE, q_scale=FAKE, cache=FAKE, cache_scale=FAKE, num_pages=4, block_table=FAKE,
+              max_pages_per_seq=4, page_size=64, seq_lens=FAKE, batch=1, q_len=1, n_heads=128, num_splits=2,
+              split_tokens=128, softmax_scale=1 / math.sqrt(192), o_part=FAKE, lse_part=FAKE, err_word=None,
+              stream=0)
+    kw.update(over)
+    return kw
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(n_heads=64), mla.MLA_ERR_UNSUPPORTED),            # the 8-bit form is the pair kernel's: 65..128 heads
+    (dict(n_heads=129), mla.MLA_ERR_UNSUPPORTED),
+    (dict(page_size=32), mla.MLA_ERR_UNSUPPORTED),
+    (dict(num_splits=1), mla.MLA_ERR_INVALID_ARG),          # 1*128 < 4*64
+    (dict(q_scale=None), mla.MLA_ERR_INVALID_ARG),
+    (dict(cache_scale=None), mla.MLA_ERR_INVALID_ARG),
+    (dict(cache_scale=FAKE + 4), mla.MLA_ERR_INVALID_ARG),   # scales read as float4
+    (dict(q8=FAKE + 8), mla.MLA_ERR_INVALID_ARG),
+    (dict(softmax_scale=0.0), mla.MLA_ERR_INVALID_ARG),
+    (dict(batch=40000, q_len=2), mla.MLA_ERR_UNSUPPORTED),   # more than 65535 query rows
+])
+def test_decode_q8_validation(lib, over, status):
+    with pytest.raises(mla.MlaError) as e:
+        mla.mla_decode_fwd_q8(**_q8_kwargs(**over))
+    assert e.value.status == status
+    assert lib.mla_last_error_message().decode().startswith("mla_decode_fwd_q8")
+
+
+def test_split_q_validation(lib):
+    with pytest.raises(mla.MlaError) as e:
+        mla.mla_split_q_e4m3(FAKE, 4, 0, FAKE, FAKE, 0)
+    assert e.value.status == mla.MLA_ERR_INVALID_ARG
+    with pytest.raises(mla.MlaError) as e:
+        mla.mla_split_q_e4m3(FAKE, 4, 128, None, FAKE, 0)
+    assert e.value.status == mla.MLA_ERR_INVALID_ARG
+    with pytest.raises(mla.MlaError) as e:
+        mla.mla_split_q_e4m3(FAKE + 2, 4, 128, FAKE, FAKE, 0)
+    assert e.value.status == mla.MLA_ERR_INVALID_ARG
+    mla.mla_split_q_e4m3(None, 0, 128, None, None, 0)        # zero rows: nothing enqueued

@@ -45,3 +45,25 @@ def test_e4m3_mtp_workload_is_tensor_bound():
     assert r["achieved"] == pytest.approx(f / 0.8e-3 / 1e12)
     assert r["frac"] == pytest.approx(r["achieved"] / PEAKS["bf16_tflops"])
     assert r["algorithmic_bytes_per_launch"] == b and r["algorithmic_flops_per_launch"] == f
+
+
+def test_e4m3_operands_take_twice_the_bf16_peak():
+    import bench
+    b, f = _units("fp8_mtp")
+    r = bench.binding_roofline(b, f, 0.3, PEAKS, None, "e4m3")
+    assert r["bound"] == "tensor" and r["mma"] == "e4m3"
+    assert r["peak"] == pytest.approx(2 * PEAKS["bf16_tflops"])
+    assert r["frac"] == pytest.approx(f / 0.3e-3 / 1e12 / (2 * PEAKS["bf16_tflops"]))
+    s = bench._decode_summary(b, f, 0.3, 0.4, PEAKS, "e4m3")
+    assert s["tensor_frac_burst"] == pytest.approx(r["frac"])
+
+
+def test_mma_type_of_a_step():
+    import bench
+
+    class Step:
+        def __init__(self, q8, cache_dtype):
+            self.q8, self.cache_dtype = q8, cache_dtype
+    assert bench.mma_type(Step(True, 2)) == "e4m3"
+    assert bench.mma_type(Step(False, 2)) == "f16"
+    assert bench.mma_type(Step(False, 1)) == "bf16"
