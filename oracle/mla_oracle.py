@@ -40,6 +40,10 @@ Readings where the pages are silent:
     at column h*128 + i; W_kv,a is [576, d].
   * e4m3 cache: one fp32 scale per token over all 576 values, scale = a/448
     with a = max |x|; code = RNE-satfinite(x * 448 / a); a = 0 -> all zero.
+  * 8-bit tensor-core MMAs over an e4m3 cache take the query as two e4m3
+    terms on one fp32 scale per (row, head) (split_query_e4m3); the pages
+    fix no such encoding, and the attention itself is still checked against
+    the exact formulas above.
 """
 from __future__ import annotations
 
