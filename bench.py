@@ -67,7 +67,8 @@ def binding_roofline(alg_bytes, alg_flops, launch_ms, pk, traffic, mma="bf16"):
     if alg_flops / (tpk * 1e12) > alg_bytes / (pk["hbm_gbs"] * 1e9):
         achieved = alg_flops / s / 1e12
         r = {"bound": "tensor", "achieved": achieved, "peak": tpk, "unit": "TFLOP/s",
-             "frac": achieved / tpk, "traffic": traffic, "mma": mma}
+             "frac": achieved / tpk, "traffic": traffic, "mma": mma,
+             "frac_of_bf16_peak": achieved / pk["bf16_tflops"]}
     else:
         achieved = alg_bytes / s / 1e9
         r = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",

@@ -53,6 +53,7 @@ def test_e4m3_operands_take_twice_the_bf16_peak():
     r = bench.binding_roofline(b, f, 0.3, PEAKS, None, "e4m3")
     assert r["bound"] == "tensor" and r["mma"] == "e4m3"
     assert r["peak"] == pytest.approx(2 * PEAKS["bf16_tflops"])
+    assert r["frac_of_bf16_peak"] == pytest.approx(2 * r["frac"])
     assert r["frac"] == pytest.approx(f / 0.3e-3 / 1e12 / (2 * PEAKS["bf16_tflops"]))
     s = bench._decode_summary(b, f, 0.3, 0.4, PEAKS, "e4m3")
     assert s["tensor_frac_burst"] == pytest.approx(r["frac"])
