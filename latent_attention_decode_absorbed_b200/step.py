@@ -5,7 +5,8 @@ rope tables, workspace and outputs, as torch tensors) and runs
 
     mla_cache_append -> mla_absorb_q -> mla_decode_fwd -> mla_combine -> mla_out_uv
 
-on one stream.  It only allocates and marshals; every step runs in libmla.
+on one stream (over an e4m3 cache with 65..128 heads: mla_absorb_q then
+mla_split_q_e4m3, and mla_decode_fwd_q8 for the attention).  It only allocates and marshals; every step runs in libmla.
 ``DecodeStep.capture`` records the same calls as CUDA graphs, for steps whose
 device work is shorter than the host time of five marshalled calls.
 """
@@ -31,7 +32,10 @@ class DecodeStep:
     """Device state of one layer for `batch` sequences with `q_len` new tokens.
 
     block_table: int32 [batch, max_pages] (host array or tensor); num_pages:
-    size of the page pool; split_tokens: split-KV chunk (multiple of 64)."""
+    size of the page pool; split_tokens: split-KV chunk (multiple of 64).
+    q8: with an e4m3 cache, bf16 queries and 65..128 heads the attention runs
+    on 8-bit MMAs (mla_split_q_e4m3 in absorb, mla_decode_fwd_q8 in attend)
+    unless q8=False, which keeps mla_decode_fwd's widened f16 operands."""
 
     def __init__(self, *, batch, q_len, n_heads, dtype, cache_dtype, block_table, num_pages,
                  split_tokens, max_pos=None, theta=10000.0, eps=1e-6, norm_gain=None,
