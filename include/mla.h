@@ -246,7 +246,8 @@ mla_status mla_decode_fwd(const void* q_abs, mla_dtype q_dtype, const void* cach
  *   q8[r, 1, h, :] = e4m3(y - hi)         (lo; y - hi is exact)
  *   q_scale[r, h]  = a / 448
  * so that q_abs ~ q_scale * (hi + lo) to about 2^-8 relative.
- *   q_abs   device bf16 [rows, n_heads, 576]  (16-byte aligned)
+ *   q_abs   device bf16 [rows, n_heads, 576]  (16-byte aligned; finite values: an infinite
+ *           one turns the whole vector's codes into NaN)
  *   q8      device uint8 [rows, 2, n_heads, 576] e4m3 codes (16-byte aligned), caller-owned
  *   q_scale device float [rows, n_heads], caller-owned
  * rows >= 0 (0 is a no-op), 1 <= n_heads <= 128.

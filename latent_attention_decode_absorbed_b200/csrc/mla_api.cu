@@ -204,8 +204,8 @@ mla_status mla_decode_fwd_q8(const void* q8, const float* q_scale, const void* c
               "mla_decode_fwd_q8: softmax_scale must be finite and > 0");
   MLA_REQUIRE(q8 && q_scale && cache && cache_scale && block_table && seq_lens && o_part && lse_part,
               MLA_ERR_INVALID_ARG, "mla_decode_fwd_q8: null pointer");
-  MLA_REQUIRE(aligned(q8, 16) && aligned(cache, 128) && aligned(o_part, 16) && aligned(cache_scale, 16),
-              MLA_ERR_INVALID_ARG, "mla_decode_fwd_q8: q8, cache_scale and o_part must be 16-byte aligned, cache 128-byte aligned");
+  MLA_REQUIRE(aligned(q8, 16) && aligned(cache, 128) && aligned(o_part, 16), MLA_ERR_INVALID_ARG,
+              "mla_decode_fwd_q8: q8 and o_part must be 16-byte aligned, cache 128-byte aligned");
   MLA_REQUIRE((long long)batch * q_len <= 65535, MLA_ERR_UNSUPPORTED, "mla_decode_fwd_q8: batch*q_len above 65535");
   DecodeArgs a{q8, MLA_E4M3, cache, cache_scale, MLA_E4M3, num_pages, block_table, max_pages_per_seq,
                page_size, seq_lens, batch, q_len, n_heads, num_splits, split_tokens, softmax_scale,

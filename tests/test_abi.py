@@ -172,7 +172,6 @@ def _q8_kwargs(**over):
     (dict(num_splits=1), mla.MLA_ERR_INVALID_ARG),          # 1*128 < 4*64
     (dict(q_scale=None), mla.MLA_ERR_INVALID_ARG),
     (dict(cache_scale=None), mla.MLA_ERR_INVALID_ARG),
-    (dict(cache_scale=FAKE + 4), mla.MLA_ERR_INVALID_ARG),   # scales read as float4
     (dict(q8=FAKE + 8), mla.MLA_ERR_INVALID_ARG),
     (dict(softmax_scale=0.0), mla.MLA_ERR_INVALID_ARG),
     (dict(batch=40000, q_len=2), mla.MLA_ERR_UNSUPPORTED),   # more than 65535 query rows
