@@ -25,6 +25,8 @@
  *   mla_cache_append  new kv_a rows -> cache rows (RMSNorm, RoPE, cast/quantise)
  *   mla_absorb_q      q_nope, q_pe  -> q_abs = [W_UK^T q_nope ; q_pe]   (576 per head)
  *   mla_decode_fwd    q_abs, cache  -> split-KV partials (o_part, lse_part)
+ *   (over an e4m3 cache with 65..128 heads, on 8-bit MMAs: mla_split_q_e4m3
+ *    q_abs -> two-term e4m3 query, then mla_decode_fwd_q8 -> the same partials)
  *   mla_combine       partials      -> o_lat (512 per head), lse
  *   (mla_combine_shards: the same merge over the per-GPU results of sequences
  *    whose cached rows are sharded across GPUs)
